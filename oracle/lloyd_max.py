@@ -82,6 +82,9 @@ def _solve(b: int):
                    c, xtol=1e-15)
     for _ in range(20):
         c = centroids_for_thresholds(thresholds_for_centroids(c))
+    # N(0,1) is symmetric, so the optimal quantizer is: c_k = -c_{N-1-k}
+    # (makes the middle threshold exactly 0 instead of a rounding residue)
+    c = 0.5 * (c - c[::-1])
     t = thresholds_for_centroids(c)
     p = cell_probability(np.concatenate([[-np.inf], t]), np.concatenate([t, [np.inf]]))
     d = 1.0 - float(np.sum(p * c * c))
