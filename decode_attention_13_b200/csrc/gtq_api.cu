@@ -1,0 +1,252 @@
+// C ABI of libgtq: argument validation, plan lifetime and kernel launches.
+// Every entry point returns a GTQ_* code; nothing throws across the boundary.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "gtq_internal.h"
+
+using namespace gtq;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_config(const gtq_config* c, bool need_128) {
+  if (!c) return GTQ_ERR_INVALID;
+  if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1) return GTQ_ERR_INVALID;
+  if (c->n_q_heads % c->n_kv_heads) return GTQ_ERR_INVALID;
+  if (c->n_q_heads / c->n_kv_heads > kMaxGq) return GTQ_ERR_UNSUPPORTED;
+  if (c->head_dim < 4 || c->head_dim > kD || (c->head_dim & 1)) return GTQ_ERR_UNSUPPORTED;
+  if (need_128 && c->head_dim != kD) return GTQ_ERR_UNSUPPORTED;
+  if (c->max_bits < 1 || c->max_bits > GTQ_MAX_BITS) return GTQ_ERR_INVALID;
+  if (c->k_bits < 1 || c->k_bits > c->max_bits) return GTQ_ERR_INVALID;
+  if (c->v_bits < 1 || c->v_bits > GTQ_MAX_BITS) return GTQ_ERR_INVALID;
+  if (c->rope_pairing != GTQ_PAIRING_HALF && c->rope_pairing != GTQ_PAIRING_INTERLEAVED)
+    return GTQ_ERR_INVALID;
+  if (c->in_dtype != GTQ_DTYPE_FP16 && c->in_dtype != GTQ_DTYPE_FP32) return GTQ_ERR_INVALID;
+  if (c->reserved != 0) return GTQ_ERR_INVALID;
+  if (c->t_capacity < 1 || c->t_capacity > (int64_t(1) << 40)) return GTQ_ERR_INVALID;
+  return GTQ_OK;
+}
+
+int cuda_code(cudaError_t e) {
+  if (e == cudaSuccess) return GTQ_OK;
+  return e == cudaErrorMemoryAllocation ? GTQ_ERR_OOM : GTQ_ERR_CUDA;
+}
+
+void release(gtq_plan* p) {
+  if (!p) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->device);
+  cudaFree(p->d_energy);
+  cudaFree(p->d_bits);
+  cudaFree(p->d_meta);
+  cudaFree(p->d_mrow);
+  cudaFree(p->d_qrot);
+  cudaFree(p->d_partials);
+  cudaFree(p->d_tickets);
+  cudaFree(p->d_status);
+  cudaSetDevice(prev);
+  delete p;
+}
+
+// common plan construction: validation done by the caller
+int make_plan(const gtq_config* cfg, gtq_plan** out) {
+  gtq_plan* p = new (std::nothrow) gtq_plan();
+  if (!p) return GTQ_ERR_OOM;
+  p->cfg = *cfg;
+  if (cudaGetDevice(&p->device) != cudaSuccess) {
+    delete p;
+    return GTQ_ERR_CUDA;
+  }
+  cudaDeviceGetAttribute(&p->n_sms, cudaDevAttrMultiProcessorCount, p->device);
+  p->n_heads = cfg->batch * cfg->n_kv_heads;
+  p->n_blocks = cfg->head_dim / 2;
+  p->g_q = cfg->n_q_heads / cfg->n_kv_heads;
+  p->n_tiles = (cfg->t_capacity + kTile - 1) / kTile;
+  p->tile_bytes = gtq_layout_tile_bytes(cfg->k_bits, cfg->v_bits);
+  p->packed_bytes = (size_t)p->n_heads * p->n_tiles * p->tile_bytes;
+  int rc = tables_for(p->device, cfg->seed, &p->tab);
+  if (rc != GTQ_OK) {
+    delete p;
+    return rc;
+  }
+  const size_t H = p->n_heads;
+  cudaError_t e = cudaSuccess;
+  auto alloc = [&](void** ptr, size_t bytes) {
+    if (e == cudaSuccess) e = cudaMalloc(ptr, bytes);
+  };
+  alloc((void**)&p->d_energy, H * p->n_blocks * sizeof(double));
+  alloc((void**)&p->d_bits, H * p->n_blocks);
+  alloc((void**)&p->d_meta, H * sizeof(HeadMeta));
+  alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
+  alloc((void**)&p->d_qrot, H * 8 * kD * sizeof(float));
+  alloc((void**)&p->d_partials, H * kMaxSplits * 8 * kPartialStride * sizeof(float));
+  alloc((void**)&p->d_tickets, H * sizeof(unsigned));
+  alloc((void**)&p->d_status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(p->d_meta, 0, H * sizeof(HeadMeta));
+  if (e != cudaSuccess) {
+    release(p);
+    return cuda_code(e);
+  }
+  *out = p;
+  return GTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gtq_layout_tile_bytes(int32_t k_bits, int32_t v_bits) {
+  if (k_bits < 1 || k_bits > GTQ_MAX_BITS || v_bits < 1 || v_bits > GTQ_MAX_BITS) return 0;
+  return (size_t)1024 * (k_bits + v_bits) + 128 + 128 * kMaxGroups;
+}
+
+int gtq_alloc_bits(const gtq_config* cfg, const void* k_dev, int64_t T, const int64_t k_strides[4],
+                   void* stream, gtq_plan** out) {
+  if (!out || !k_dev || !k_strides) return GTQ_ERR_INVALID;
+  int rc = check_config(cfg, false);
+  if (rc != GTQ_OK) return rc;
+  if (cfg->head_dim % 8) return GTQ_ERR_UNSUPPORTED;  // energy pass reads 8-dim vectors
+  if (T < 1 || T > cfg->t_capacity) return GTQ_ERR_INVALID;
+  const int esz = cfg->in_dtype == GTQ_DTYPE_FP16 ? 2 : 4;
+  if (k_strides[3] != 1 || !aligned(k_dev, 16)) return GTQ_ERR_INVALID;
+  for (int i = 0; i < 3; ++i)
+    if (k_strides[i] < 0 || (k_strides[i] * esz) % 16) return GTQ_ERR_INVALID;
+  gtq_plan* p = nullptr;
+  rc = make_plan(cfg, &p);
+  if (rc != GTQ_OK) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_energy(p, k_dev, T, k_strides, s);
+  if (e == cudaSuccess) e = launch_greedy_and_meta(p, s);
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(s);
+    release(p);
+    return cuda_code(e);
+  }
+  *out = p;
+  return GTQ_OK;
+}
+
+int gtq_alloc_bits_from_energy(const gtq_config* cfg, const double* host_energy, gtq_plan** out) {
+  if (!out || !host_energy) return GTQ_ERR_INVALID;
+  int rc = check_config(cfg, false);
+  if (rc != GTQ_OK) return rc;
+  gtq_plan* p = nullptr;
+  rc = make_plan(cfg, &p);
+  if (rc != GTQ_OK) return rc;
+  cudaError_t e = cudaMemcpy(p->d_energy, host_energy,
+                             (size_t)p->n_heads * p->n_blocks * sizeof(double),
+                             cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = launch_greedy_and_meta(p, 0);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+  if (e != cudaSuccess) {
+    release(p);
+    return cuda_code(e);
+  }
+  *out = p;
+  return GTQ_OK;
+}
+
+int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_dev,
+                      const int64_t strides[4], int64_t t0, int64_t n_tokens, void* packed_dev,
+                      size_t packed_bytes, void* stream) {
+  if (!plan || !k_dev || !v_dev || !strides || !packed_dev) return GTQ_ERR_INVALID;
+  if (plan->cfg.head_dim != kD) return GTQ_ERR_UNSUPPORTED;
+  if (t0 < 0 || n_tokens < 1 || t0 + n_tokens > plan->cfg.t_capacity) return GTQ_ERR_INVALID;
+  if (packed_bytes < plan->packed_bytes || !aligned(packed_dev, 16)) return GTQ_ERR_INVALID;
+  const int esz = plan->cfg.in_dtype == GTQ_DTYPE_FP16 ? 2 : 4;
+  if (strides[3] != 1 || !aligned(k_dev, esz) || !aligned(v_dev, esz)) return GTQ_ERR_INVALID;
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] < 0) return GTQ_ERR_INVALID;
+  return cuda_code(launch_quantize(plan, k_dev, v_dev, strides, t0, n_tokens,
+                                   (uint8_t*)packed_dev, (cudaStream_t)stream));
+}
+
+int gtq_decode_attn(gtq_plan* plan, const void* packed_dev, int64_t T, const void* q_dev,
+                    int32_t q_dtype, float* out_dev, void* stream) {
+  if (!plan || !packed_dev || !q_dev || !out_dev) return GTQ_ERR_INVALID;
+  if (plan->cfg.head_dim != kD) return GTQ_ERR_UNSUPPORTED;
+  if (T < 1 || T > plan->cfg.t_capacity) return GTQ_ERR_INVALID;
+  if (q_dtype != GTQ_DTYPE_FP16 && q_dtype != GTQ_DTYPE_FP32) return GTQ_ERR_INVALID;
+  if (!aligned(packed_dev, 16) || !aligned(q_dev, 16) || !aligned(out_dev, 16))
+    return GTQ_ERR_INVALID;
+  return cuda_code(launch_decode(plan, (const uint8_t*)packed_dev, T, q_dev, q_dtype, out_dev,
+                                 (cudaStream_t)stream));
+}
+
+int gtq_free(gtq_plan* plan) {
+  if (!plan) return GTQ_OK;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(plan->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaSetDevice(prev);
+  release(plan);
+  return cuda_code(e);
+}
+
+size_t gtq_packed_bytes(const gtq_plan* plan) { return plan ? plan->packed_bytes : 0; }
+
+int gtq_get_bits(gtq_plan* plan, uint8_t* host_bits, void* stream) {
+  if (!plan || !host_bits) return GTQ_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(host_bits, plan->d_bits, (size_t)plan->n_heads * plan->n_blocks,
+                                  cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_code(e);
+}
+
+int gtq_get_energy(gtq_plan* plan, double* host_energy, void* stream) {
+  if (!plan || !host_energy) return GTQ_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(host_energy, plan->d_energy,
+                                  (size_t)plan->n_heads * plan->n_blocks * sizeof(double),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_code(e);
+}
+
+int gtq_status(gtq_plan* plan) {
+  if (!plan) return GTQ_ERR_INVALID;
+  int v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, plan->d_status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(plan->d_status, 0, sizeof(int));
+  if (e != cudaSuccess) return GTQ_ERR_CUDA;
+  if (v & kStatusTimeout) return GTQ_ERR_TIMEOUT;
+  if (v & kStatusOverflow) return GTQ_ERR_OVERFLOW;
+  return GTQ_OK;
+}
+
+const char* gtq_strerror(int code) {
+  switch (code) {
+    case GTQ_OK: return "ok";
+    case GTQ_ERR_INVALID: return "invalid argument";
+    case GTQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GTQ_ERR_CUDA: return "CUDA runtime error";
+    case GTQ_ERR_OOM: return "device out of memory";
+    case GTQ_ERR_TIMEOUT: return "bounded device wait expired";
+    case GTQ_ERR_OVERFLOW: return "norm above the fp16 range (clamped)";
+    case GTQ_ERR_STATE: return "plan not ready";
+    default: return "unknown error";
+  }
+}
+
+int gtq_lloyd_max(int32_t bits, double* centroids, double* thresholds, double* distortion) {
+  return lloyd_max_host(bits, centroids, thresholds, distortion);
+}
+
+int gtq_rotation(uint64_t seed, int32_t tag, int32_t m, double* out) {
+  if (tag != 0x4B && tag != 0x56) return GTQ_ERR_INVALID;
+  if (tag == 0x4B && (m < 2 || m > kD || (m & 1))) return GTQ_ERR_INVALID;
+  if (tag == 0x56 && m != kD) return GTQ_ERR_INVALID;
+  return rotation_host(seed, tag, m, out);
+}
+
+}  // extern "C"

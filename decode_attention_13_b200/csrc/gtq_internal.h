@@ -1,0 +1,108 @@
+// Internal declarations of libgtq (not part of the C ABI).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gtq.h"
+
+namespace gtq {
+
+constexpr int kTile = GTQ_TILE_TOKENS;  // tokens per packed tile
+constexpr int kD = 128;                 // head_dim of quantize / decode
+constexpr int kBlocks = kD / 2;         // RoPE blocks per head
+constexpr int kMaxGroups = 8;           // one group per nonzero width 1..8
+constexpr int kMaxSegs = 16;            // (k-tile, group) intersections <= 8 + 8 - 1
+constexpr int kMaxGq = 8;               // query heads per KV head handled by decode
+constexpr int kLutEntries = 510;        // sum over w = 1..8 of 2^w
+constexpr int kThrEntries = 502;        // sum over w = 1..8 of (2^w - 1)
+constexpr int kMaxSplits = 256;         // context splits per head in decode
+constexpr int kPartialStride = 2 + kD;  // (m, l, o[128]) per (split, q head)
+constexpr int kStatusOverflow = 1;      // status word bits
+constexpr int kStatusTimeout = 2;
+
+// First LUT / threshold entry of width w (1..8).
+__host__ __device__ inline int lut_base(int w) { return (1 << w) - 2; }
+__host__ __device__ inline int thr_base(int w) { return (1 << w) - 1 - w; }
+
+// Per-head metadata derived from the allocation (built on the device).
+struct HeadMeta {
+  int32_t n_groups;  // G_K: nonzero-width groups
+  int32_t n_slots;   // sum over groups of m/2
+  int32_t n_ktiles;  // ceil(n_slots / 8)
+  int32_t n_segs;    // (k-tile, group) segments
+  float inv_sqrt_m[kMaxGroups];
+  float sqrt_m[kMaxGroups];
+  uint8_t grp_width[kMaxGroups];  // descending
+  uint8_t grp_m[kMaxGroups];
+  uint8_t grp_first_slot[kMaxGroups];
+  uint8_t grp_split[kMaxGroups];  // decode computes this group's logits in split fp16
+  uint8_t slot_width[kBlocks];
+  uint8_t slot_group[kBlocks];
+  uint16_t slot_koff[kBlocks];    // byte offset of the slot in the key-code area
+  uint8_t block_group[kBlocks];   // group of each RoPE block (0xFF: width 0)
+  uint8_t kt_seg_start[8];
+  uint8_t kt_seg_count[8];
+  uint8_t seg_group[kMaxSegs];
+  uint8_t seg_lo[kMaxSegs];       // slot range [lo, hi) within the k-tile (0..8)
+  uint8_t seg_hi[kMaxSegs];
+  uint8_t seg_last[kMaxSegs];     // the group ends in this segment
+};
+
+// Device-resident constant tables shared by every plan of a (device, seed).
+struct Tables {
+  double* rot_k;     // R_m for m = 2, 4, ..., 128, row-major, concatenated (fp64)
+  float* rot_v;      // R_V 128 x 128 row-major (fp32)
+  double* dist;      // D(0..8)
+  float* thr;        // fp32 thresholds, width w at thr_base(w)
+  __half* lut_hi;    // fp16(centroid), width w at lut_base(w)
+  __half* lut_lo;    // fp16(centroid - fp16(centroid))
+};
+
+inline size_t rot_k_offset(int m) {  // element offset of R_m (m even) in rot_k
+  size_t off = 0;
+  for (int mm = 2; mm < m; mm += 2) off += (size_t)mm * mm;
+  return off;
+}
+inline size_t rot_k_total() { return rot_k_offset(kD + 2); }
+
+}  // namespace gtq
+
+// Opaque plan (C ABI type).
+struct gtq_plan {
+  gtq_config cfg;
+  int device;
+  int n_heads;        // batch * n_kv_heads
+  int n_blocks;       // head_dim / 2
+  int g_q;            // n_q_heads / n_kv_heads
+  int64_t n_tiles;    // tiles per head (capacity)
+  size_t tile_bytes;
+  size_t packed_bytes;
+  int n_sms;
+  gtq::Tables tab;    // borrowed from the library cache (not freed by the plan)
+  double* d_energy;   // [heads][n_blocks]
+  uint8_t* d_bits;    // [heads][n_blocks]
+  gtq::HeadMeta* d_meta;  // [heads]
+  float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
+  float* d_qrot;      // [heads][8][128] rotated, scaled queries (decode workspace)
+  float* d_partials;  // [heads][kMaxSplits][8][kPartialStride]
+  unsigned* d_tickets;  // [heads]
+  int* d_status;      // device status word
+};
+
+namespace gtq {
+// Host tables (gtq_tables.cu)
+int lloyd_max_host(int bits, double* c, double* t, double* d);
+int rotation_host(uint64_t seed, int tag, int m, double* out);
+int tables_for(int device, uint64_t seed, Tables* out);  // cached per (device, seed)
+
+// Kernel launchers
+cudaError_t launch_energy(const gtq_plan* p, const void* k, int64_t T, const int64_t* st,
+                          cudaStream_t s);
+cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s);
+cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                            int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s);
+cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, const void* q,
+                          int q_dtype, float* out, cudaStream_t s);
+}  // namespace gtq

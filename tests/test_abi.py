@@ -1,0 +1,116 @@
+"""CPU checks of the C ABI (no GPU calls): the library loads, exports every
+function include/gtq.h declares, its host tables match the oracle, and
+argument validation rejects bad calls before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import decode_attention_13_b200 as gtq
+from oracle import lloyd_max, rotation
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "gtq.h")).read()
+    return set(re.findall(r"GTQ_API\s+[\w\s\*]+?\b(gtq_\w+)\s*\(", text))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == set(gtq.binding.ABI_FUNCTIONS)
+
+
+def test_every_declared_symbol_exported():
+    lib = ctypes.CDLL(gtq.binding.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_library_lloyd_max_matches_oracle():
+    for b in range(0, 9):
+        c, t, d = gtq.gtq_lloyd_max(b)
+        assert np.max(np.abs(c - lloyd_max.centroids(b))) < 1e-12
+        if b:
+            assert np.max(np.abs(t - lloyd_max.thresholds(b))) < 1e-12
+            assert np.array_equal(t.astype(np.float32), lloyd_max.thresholds(b).astype(np.float32))
+        assert abs(d - lloyd_max.distortion(b)) < 1e-15
+
+
+def test_library_rotations_match_oracle():
+    for seed in (0, 7):
+        for m in (2, 4, 18, 64, 128):
+            assert np.max(np.abs(gtq.gtq_rotation(m, gtq.TAG_KEY, seed) - rotation.key_rotation(m, seed))) < 1e-12
+        assert np.max(np.abs(gtq.gtq_rotation(128, gtq.TAG_VALUE, seed) - rotation.value_rotation(128, seed))) < 1e-12
+
+
+def test_tile_bytes():
+    assert gtq.gtq_layout_tile_bytes(3, 3) == 1024 * 6 + 128 + 1024
+    assert gtq.gtq_layout_tile_bytes(0, 3) == 0
+
+
+def _cfg(**kw):
+    base = dict(batch=1, n_q_heads=8, n_kv_heads=2, k_bits=3, v_bits=3, t_capacity=1024)
+    base.update(kw)
+    return gtq.make_config(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), gtq.GTQ_ERR_INVALID),
+    (dict(n_q_heads=7), gtq.GTQ_ERR_INVALID),
+    (dict(n_q_heads=18), gtq.GTQ_ERR_UNSUPPORTED),      # GQA group of 9
+    (dict(head_dim=130), gtq.GTQ_ERR_UNSUPPORTED),
+    (dict(head_dim=12), gtq.GTQ_ERR_UNSUPPORTED),       # alloc from K needs a multiple of 8
+    (dict(k_bits=0), gtq.GTQ_ERR_INVALID),
+    (dict(k_bits=9), gtq.GTQ_ERR_INVALID),
+    (dict(v_bits=9), gtq.GTQ_ERR_INVALID),
+    (dict(rope_pairing=2), gtq.GTQ_ERR_INVALID),
+    (dict(in_dtype=3), gtq.GTQ_ERR_INVALID),
+    (dict(t_capacity=0), gtq.GTQ_ERR_INVALID),
+])
+def test_alloc_rejects_bad_config(kw, code):
+    cfg = _cfg(**kw)
+    st = (ctypes.c_int64 * 4)(2 * 1024 * 128, 1024 * 128, 128, 1)
+    out = ctypes.c_void_p()
+    rc = gtq.binding._lib.gtq_alloc_bits(ctypes.byref(cfg), 0x1000, 16, st, None, ctypes.byref(out))
+    assert rc == code and out.value is None
+
+
+def test_alloc_rejects_bad_pointers_and_sizes():
+    lib = gtq.binding._lib
+    cfg = _cfg()
+    st = (ctypes.c_int64 * 4)(2 * 1024 * 128, 1024 * 128, 128, 1)
+    out = ctypes.c_void_p()
+    assert lib.gtq_alloc_bits(None, 0x1000, 16, st, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_alloc_bits(ctypes.byref(cfg), None, 16, st, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_alloc_bits(ctypes.byref(cfg), 0x1002, 16, st, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_alloc_bits(ctypes.byref(cfg), 0x1000, 0, st, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_alloc_bits(ctypes.byref(cfg), 0x1000, 2048, st, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    bad = (ctypes.c_int64 * 4)(2 * 1024 * 128, 1024 * 128, 128, 2)
+    assert lib.gtq_alloc_bits(ctypes.byref(cfg), 0x1000, 16, bad, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    odd = (ctypes.c_int64 * 4)(2 * 1024 * 128, 1024 * 128, 129, 1)
+    assert lib.gtq_alloc_bits(ctypes.byref(cfg), 0x1000, 16, odd, None, ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    assert out.value is None
+
+
+def test_null_plan_calls():
+    lib = gtq.binding._lib
+    st = (ctypes.c_int64 * 4)(0, 0, 128, 1)
+    assert lib.gtq_quantize_pack(None, 0x1000, 0x1000, st, 0, 1, 0x1000, 1 << 20, None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_decode_attn(None, 0x1000, 1, 0x1000, 0, 0x1000, None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_free(None) == gtq.GTQ_OK
+    assert lib.gtq_packed_bytes(None) == 0
+    assert lib.gtq_status(None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_get_bits(None, None, None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_lloyd_max(9, None, None, None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_rotation(0, 0x4B, 3, None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_rotation(0, 0x41, 4, (ctypes.c_double * 16)()) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_rotation(0, 0x56, 64, (ctypes.c_double * 4096)()) == gtq.GTQ_ERR_INVALID
+
+
+def test_strerror_names():
+    for code in range(-7, 1):
+        assert gtq.strerror(code) and gtq.strerror(code) != "unknown error"
+    assert gtq.strerror(-99) == "unknown error"
