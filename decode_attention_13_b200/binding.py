@@ -43,14 +43,17 @@ TAG_VALUE = 0x56
 ABI_FUNCTIONS = (
     "gtq_alloc_bits", "gtq_alloc_bits_from_energy", "gtq_quantize_pack", "gtq_decode_attn",
     "gtq_free", "gtq_packed_bytes", "gtq_get_bits", "gtq_get_energy", "gtq_status",
-    "gtq_strerror", "gtq_lloyd_max", "gtq_rotation", "gtq_layout_tile_bytes",
+    "gtq_strerror", "gtq_last_error", "gtq_lloyd_max", "gtq_rotation", "gtq_layout_tile_bytes",
 )
 
 
 class GtqError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__("%s failed: %s (%d)" % (where, strerror(code), code))
+        detail = ""
+        if code in (GTQ_ERR_CUDA, GTQ_ERR_OOM):
+            detail = " [%s]" % _lib.gtq_last_error().decode()
+        super().__init__("%s failed: %s (%d)%s" % (where, strerror(code), code, detail))
 
 
 class gtq_config(ctypes.Structure):
@@ -88,6 +91,7 @@ def _load():
         "gtq_get_energy": (I32, [P, ctypes.POINTER(ctypes.c_double), P]),
         "gtq_status": (I32, [P]),
         "gtq_strerror": (ctypes.c_char_p, [I32]),
+        "gtq_last_error": (ctypes.c_char_p, []),
         "gtq_lloyd_max": (I32, [I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
         "gtq_rotation": (I32, [ctypes.c_uint64, I32, I32, ctypes.POINTER(ctypes.c_double)]),
         "gtq_layout_tile_bytes": (SZ, [I32, I32]),

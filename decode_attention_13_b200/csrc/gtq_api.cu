@@ -1,6 +1,7 @@
 // C ABI of libgtq: argument validation, plan lifetime and kernel launches.
 // Every entry point returns a GTQ_* code; nothing throws across the boundary.
 #include <algorithm>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -31,8 +32,12 @@ int check_config(const gtq_config* c, bool need_128) {
   return GTQ_OK;
 }
 
+thread_local char g_last_error[256] = "";
+
 int cuda_code(cudaError_t e) {
   if (e == cudaSuccess) return GTQ_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
   return e == cudaErrorMemoryAllocation ? GTQ_ERR_OOM : GTQ_ERR_CUDA;
 }
 
@@ -223,6 +228,8 @@ int gtq_status(gtq_plan* plan) {
   if (v & kStatusOverflow) return GTQ_ERR_OVERFLOW;
   return GTQ_OK;
 }
+
+const char* gtq_last_error(void) { return g_last_error; }
 
 const char* gtq_strerror(int code) {
   switch (code) {

@@ -51,6 +51,9 @@ struct QuantSmem {
   int overflow;
 };
 
+// the tile image follows QuantSmem, rounded up so that 16-byte accesses are aligned
+constexpr size_t kImgOffset = (sizeof(QuantSmem) + 127) & ~size_t(127);
+
 __device__ inline int lm_code(float y, const float* thr, int w) {
   const float* t = thr + thr_base(w);
   int lo = 0;
@@ -119,7 +122,7 @@ template <typename T>
 __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   QuantSmem& s = *reinterpret_cast<QuantSmem*>(smem_raw);
-  uint8_t* img = smem_raw + sizeof(QuantSmem);  // tile image, a.tile_bytes
+  uint8_t* img = smem_raw + kImgOffset;  // tile image, a.tile_bytes (16-byte accesses)
   uint32_t* img32 = reinterpret_cast<uint32_t*>(img);
   const int head = blockIdx.y, b = head / a.hkv, h = head % a.hkv;
   const int tid = threadIdx.x;
@@ -285,7 +288,7 @@ cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, con
   a.kb = p->cfg.k_bits;
   a.vb = p->cfg.v_bits;
   a.status = p->d_status;
-  const size_t smem = sizeof(QuantSmem) + p->tile_bytes;
+  const size_t smem = kImgOffset + p->tile_bytes;
   const int64_t tiles = (t0 + n - 1) / kTile - t0 / kTile + 1;
   int per_head = (int)std::min<int64_t>(tiles, std::max(1, (p->n_sms + p->n_heads - 1) / p->n_heads));
   dim3 grid(per_head, p->n_heads);

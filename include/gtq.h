@@ -138,7 +138,7 @@ GTQ_API int gtq_alloc_bits_from_energy(const gtq_config* cfg, const double* host
  *   k_dev, v_dev  post-RoPE K and V, in_dtype, laid out like gtq_alloc_bits'
  *                 k_dev with the same 4 strides (strides[3] == 1); token t of
  *                 the cache is row t of these tensors.
- *   packed_dev    the packed cache, >= gtq_packed_bytes(plan) bytes, 256-byte
+ *   packed_dev    the packed cache, >= gtq_packed_bytes(plan) bytes, 16-byte
  *                 aligned, caller-owned.  Tokens outside [t0, t0+n) keep their
  *                 bytes (appending to an existing cache is allowed).
  *   packed_bytes  size of packed_dev in bytes.
@@ -192,6 +192,10 @@ GTQ_API int gtq_status(gtq_plan* plan);
 
 /* Human-readable name of a return code (static string). */
 GTQ_API const char* gtq_strerror(int code);
+
+/* Name and text of the last CUDA error an entry point of this thread turned
+ * into GTQ_ERR_CUDA / GTQ_ERR_OOM ("" if none); valid until the next call. */
+GTQ_API const char* gtq_last_error(void);
 
 /* Library's own tables, computed on the host (no GPU needed):
  * the b-bit Lloyd-Max quantizer of N(0,1) (b = 0..8): 2^b centroids

@@ -1,0 +1,230 @@
+"""GPU parity of libgtq against the fp64 oracle, through the C ABI.
+
+Tolerances (the construction's match criteria):
+  * allocations: bit-exact;
+  * energies: relative 1e-12 (fp64 sums in a different order);
+  * codes: bit-exact except at most 1e-4 of them one level off -- the GPU takes
+    the threshold decision in fp32 on an fp32 rotation, the oracle rounds its
+    fp64 value to fp32 before the same decision, so only values within fp32
+    rounding of a threshold can differ;
+  * stored fp16 norms: bit-exact except at most 1e-4 of them one ulp off (fp64
+    sums in another order);
+  * decode outputs: relative L2 <= 2e-3 on identical packed inputs (the oracle's
+    codes written into the layout by tests/layout.py).
+"""
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import decode_attention_13_b200 as gtq  # noqa: E402
+from decode_attention_13_b200 import synth  # noqa: E402
+from oracle import allocation, attention, lloyd_max, quantize  # noqa: E402
+from tests import layout  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+CODE_FLIP_MAX = 1e-4
+NORM_ULP_MAX = 1e-4
+DECODE_REL_L2 = 2e-3
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(np.asarray(a, np.float64) - b) / np.linalg.norm(b))
+
+
+class Case:
+    """One layer run through the library, with the oracle's view of every head."""
+
+    def __init__(self, B, hkv, gq, T, kb, vb, pairing=0, dtype="fp16", seed=0, theta=1e4,
+                 cap=None, decay=None):
+        self.B, self.hkv, self.gq, self.T, self.kb, self.vb = B, hkv, gq, T, kb, vb
+        self.pairing = pairing
+        npdt = np.float16 if dtype == "fp16" else np.float32
+        self.lay = synth.layer((seed,), B, hkv, gq, T, theta=theta, pairing=pairing,
+                               dtype=npdt, decay=decay)
+        self.cap = cap or T
+        k = torch.zeros((B, hkv, self.cap, 128), dtype=torch.float16 if dtype == "fp16" else torch.float32)
+        v = torch.zeros_like(k)
+        k[:, :, :T] = torch.from_numpy(self.lay["k"])
+        v[:, :, :T] = torch.from_numpy(self.lay["v"])
+        self.k, self.v = k.cuda(), v.cuda()
+        self.q = torch.from_numpy(self.lay["q"]).cuda()
+        self.cfg = gtq.make_config(B, hkv * gq, hkv, kb, vb, self.cap, rope_pairing=pairing,
+                                   in_dtype=gtq.DTYPE_FP16 if dtype == "fp16" else gtq.DTYPE_FP32)
+        self.plan = gtq.gtq_alloc_bits(self.cfg, self.k, T)
+        self.packed = torch.zeros(self.plan.packed_bytes, dtype=torch.uint8, device="cuda")
+
+    def quantize(self, t0=0, n=None):
+        gtq.gtq_quantize_pack(self.plan, self.k, self.v, t0, self.T - t0 if n is None else n,
+                              self.packed)
+
+    def decode(self, packed=None):
+        out = torch.empty((self.B, self.hkv * self.gq, 128), dtype=torch.float32, device="cuda")
+        gtq.gtq_decode_attn(self.plan, self.packed if packed is None else packed, self.T, self.q, out)
+        torch.cuda.synchronize()
+        return out.cpu().numpy()
+
+    def head_bytes(self, b, h, packed=None):
+        p = (self.packed if packed is None else packed).cpu().numpy()
+        per = self.plan.packed_bytes // (self.B * self.hkv)
+        i = b * self.hkv + h
+        return p[i * per:(i + 1) * per]
+
+    # oracle side ----------------------------------------------------------
+    def oracle_head(self, b, h):
+        k = self.lay["k"][b, h]
+        e = allocation.block_energy(k, self.pairing)
+        bits = allocation.greedy_bits(e, self.kb, 128)
+        kg = quantize.quantize_keys(k, bits, self.pairing)
+        vg = quantize.quantize_values(self.lay["v"][b, h], self.vb)
+        return e, bits, kg, vg
+
+
+def compare_codes(case, b, h, kg, vg, bits):
+    keys, vcodes, vnorm = layout.read_head(case.head_bytes(b, h), bits, case.kb, case.vb, case.T)
+    by_w = {g.width: g for g in kg}
+    flips = total = nflip = ntot = 0
+    for (w, codes, n16) in keys:
+        og = by_w[w]
+        d = codes - og.codes
+        assert np.all(np.abs(d) <= 1), "code off by more than one level"
+        flips += int(np.count_nonzero(d))
+        total += d.size
+        nd = n16.view(np.uint16).astype(np.int64) - og.norm16.view(np.uint16).astype(np.int64)
+        assert np.all(np.abs(nd) <= 1)
+        nflip += int(np.count_nonzero(nd))
+        ntot += nd.size
+    d = vcodes - vg.codes
+    assert np.all(np.abs(d) <= 1)
+    flips += int(np.count_nonzero(d))
+    total += d.size
+    nd = vnorm.view(np.uint16).astype(np.int64) - vg.norm16.view(np.uint16).astype(np.int64)
+    assert np.all(np.abs(nd) <= 1)
+    nflip += int(np.count_nonzero(nd))
+    ntot += nd.size
+    assert flips <= CODE_FLIP_MAX * total, (flips, total)
+    assert nflip <= NORM_ULP_MAX * ntot, (nflip, ntot)
+    return flips, total
+
+
+def check_case(case, check_decode=True):
+    case.quantize()
+    out_gpu_e2e = case.decode()
+    bits_gpu = gtq.gtq_get_bits(case.plan)
+    e_gpu = gtq.gtq_get_energy(case.plan)
+    assert gtq.gtq_status(case.plan) == gtq.GTQ_OK
+    oracle_packed = np.zeros(case.plan.packed_bytes, np.uint8)
+    per = case.plan.packed_bytes // (case.B * case.hkv)
+    n_tiles = per // layout.tile_bytes(case.kb, case.vb)
+    ref_out = np.zeros((case.B, case.hkv * case.gq, 128))
+    for b in range(case.B):
+        for h in range(case.hkv):
+            e, bits, kg, vg = case.oracle_head(b, h)
+            assert np.allclose(e_gpu[b, h], e, rtol=1e-12, atol=0)
+            assert np.array_equal(bits_gpu[b, h].astype(np.int64), bits), (b, h)
+            compare_codes(case, b, h, kg, vg, bits)
+            q = case.lay["q"][b, h * case.gq:(h + 1) * case.gq]
+            ref_out[b, h * case.gq:(h + 1) * case.gq] = attention.decode_rotated(q, kg, vg)
+            desc = sorted(kg, key=lambda g: -g.width)
+            buf = layout.write_head(bits, [(g.width, g.codes, g.norm16) for g in desc],
+                                    vg.codes, vg.norm16, case.kb, case.vb, n_tiles)
+            i = b * case.hkv + h
+            oracle_packed[i * per:(i + 1) * per] = buf
+    if check_decode:
+        out_same_codes = case.decode(torch.from_numpy(oracle_packed).cuda())
+        assert rel_l2(out_same_codes, ref_out) <= DECODE_REL_L2
+        assert rel_l2(out_gpu_e2e, ref_out) <= DECODE_REL_L2
+    return ref_out
+
+
+@pytest.mark.parametrize("B,hkv,gq,T,kb,vb,pairing,dtype", [
+    (1, 1, 1, 1024, 3, 3, 0, "fp32"),       # the single-head fp32 correctness workload
+    (2, 2, 4, 1000, 2, 2, 0, "fp16"),
+    (1, 2, 8, 777, 3, 3, 1, "fp16"),
+    (1, 1, 7, 129, 3, 2, 0, "fp16"),
+    (1, 3, 2, 300, 4, 4, 0, "fp16"),
+    (1, 1, 8, 200, 1, 1, 0, "fp16"),
+    (1, 1, 8, 190, 8, 8, 1, "fp16"),
+    (1, 1, 5, 257, 5, 3, 0, "fp32"),
+])
+def test_layer_parity(B, hkv, gq, T, kb, vb, pairing, dtype):
+    check_case(Case(B, hkv, gq, T, kb, vb, pairing, dtype, seed=100 + T))
+
+
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129])
+def test_ragged_lengths(T):
+    check_case(Case(1, 2, 4, T, 3, 3, seed=T))
+
+
+def test_capacity_larger_than_T():
+    check_case(Case(1, 1, 8, 150, 3, 3, cap=1000, seed=5))
+
+
+def test_append_equals_one_shot():
+    one = Case(1, 2, 8, 700, 3, 3, seed=9)
+    one.quantize()
+    two = Case(1, 2, 8, 700, 3, 3, seed=9)
+    two.quantize(0, 333)
+    two.quantize(333, 1)
+    two.quantize(334, 700 - 334)
+    torch.cuda.synchronize()
+    for b in range(1):
+        for h in range(2):
+            assert np.array_equal(one.head_bytes(b, h)[: 11 * layout.tile_bytes(3, 3)],
+                                  two.head_bytes(b, h)[: 11 * layout.tile_bytes(3, 3)])
+    assert np.allclose(one.decode(), two.decode(), rtol=0, atol=0)
+
+
+def test_zero_vectors():
+    c = Case(1, 1, 4, 100, 3, 3, seed=3)
+    c.k[:, :, 10] = 0
+    c.v[:, :, 20] = 0
+    c.lay["k"][:, :, 10] = 0
+    c.lay["v"][:, :, 20] = 0
+    c.plan = gtq.gtq_alloc_bits(c.cfg, c.k, c.T)
+    check_case(c)
+
+
+def test_norm_overflow_flagged():
+    c = Case(1, 1, 1, 64, 2, 2, seed=4)
+    c.v[0, 0, 5] = 60000.0           # |v| far above 65504
+    c.quantize()
+    torch.cuda.synchronize()
+    assert gtq.gtq_status(c.plan) == gtq.GTQ_ERR_OVERFLOW
+    assert gtq.gtq_status(c.plan) == gtq.GTQ_OK   # reading clears it
+
+
+@pytest.mark.parametrize("d", [4, 6, 8, 10])
+@pytest.mark.parametrize("budget", [1, 2, 3, 4])
+def test_greedy_from_energy_tiny_heads(d, budget):
+    rng = np.random.default_rng(d * 7 + budget)
+    E = rng.exponential(1.0, (3, 2, d // 2)) * np.exp(rng.uniform(-5, 5, (3, 2, d // 2)))
+    cfg = gtq.make_config(3, 2, 2, budget, 2, 64, head_dim=d)
+    plan = gtq.gtq_alloc_bits_from_energy(cfg, E)
+    got = gtq.gtq_get_bits(plan)
+    for b in range(3):
+        for h in range(2):
+            want = allocation.greedy_bits(E[b, h], budget, d)
+            assert np.array_equal(got[b, h].astype(np.int64), want)
+
+
+def test_greedy_equal_energies_uniform():
+    for kb in (1, 2, 3, 5, 8):
+        cfg = gtq.make_config(1, 1, 1, kb, 2, 64)
+        plan = gtq.gtq_alloc_bits_from_energy(cfg, np.full((1, 1, 64), 0.25))
+        assert np.all(gtq.gtq_get_bits(plan) == kb)
+
+
+def test_greedy_ties_and_cap():
+    cfg = gtq.make_config(1, 1, 1, 4, 2, 64, head_dim=16)
+    E = np.array([[[1e12] + [1e-12] * 7]])
+    plan = gtq.gtq_alloc_bits_from_energy(cfg, E)
+    got = gtq.gtq_get_bits(plan)[0, 0].astype(np.int64)
+    assert np.array_equal(got, allocation.greedy_bits(E[0, 0], 4, 16)) and got[0] == 8
+    cfg = gtq.make_config(1, 1, 1, 3, 2, 64, head_dim=8)
+    E = np.array([[[2.0, 2.0, 1.0, 1.0]]])
+    plan = gtq.gtq_alloc_bits_from_energy(cfg, E)
+    assert np.array_equal(gtq.gtq_get_bits(plan)[0, 0].astype(np.int64),
+                          allocation.greedy_bits(E[0, 0], 3, 8))
