@@ -1,0 +1,428 @@
+"""Benchmark: packed K3V3 decode attention at 128K context on B200.
+
+Workload (default): the Qwen2.5-3B-shaped stack -- 36 layers, 16 query / 2 KV
+heads, head_dim 128, T = 131072, batch 1, K3V3 -- on synthetic fp16 K/V/q
+(seeded, RoPE theta 1e6, per-head decay and outlier blocks).  The packed cache
+of every layer is built once by the library (energy + greedy allocation +
+quantize-pack); a step is one decode over all 36 layers (query rotation,
+split-K decode, merge with R_V^T), captured in a CUDA graph.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank decodes its own independent sequence
+(weak scaling; no collective in the data path).  --impl reference times the CPU
+fp64 oracle (the method as written, never tuned) on the same workload.
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed K3V3 decode-attn cache GB/s (% HBM peak) & ctx-tokens/s at 128K"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def packed_bytes_per_token_head(kb, vb, g_k):
+    """Algorithmic bytes one decode reads per (token, KV head): key codes,
+    group norms, value codes, value norm."""
+    return 16 * kb + 2 * g_k + 16 * vb + 2
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        loaded = [x for x in sm if mx and x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- profiles
+def profile_traffic(kernel_src):
+    """dram bytes per decode launch from the committed ncu summary, or None if
+    the kernel source changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_qwen2.5-3b_128k.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    t = re.search(r"traffic_bytes_per_layer_call:\s*([0-9.eE+]+)", text)
+    if not m or not t:
+        return None
+    if m.group(1) != hashlib.sha256(open(kernel_src, "rb").read()).hexdigest():
+        return None
+    return float(t.group(1))
+
+
+# ------------------------------------------------------------ reference arm
+def oracle_pool(cfgd, n_heads=2, seed=2):
+    """A few whole KV heads of the workload, coded by the oracle (not timed)."""
+    from decode_attention_13_b200 import synth
+    from oracle import allocation, quantize
+
+    gq = cfgd["h_q"] // cfgd["h_kv"]
+    pool = []
+    for i in range(n_heads):
+        hd = synth.head((seed, 9999, i), T=cfgd["T"], theta=cfgd["theta"], g_q=gq)
+        bits = allocation.greedy_bits(allocation.block_energy(hd["k"]), cfgd["k_bits"], 128)
+        pool.append((hd["q"], quantize.quantize_keys(hd["k"], bits, 0),
+                     quantize.quantize_values(hd["v"], cfgd["v_bits"])))
+    return pool
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def oracle_decode_sample(cfgd, pool, seconds):
+    """Time the fp64 oracle's decode of whole KV heads from `pool` until
+    `seconds` elapse; returns (GB/s of packed cache, heads decoded, seconds)."""
+    from oracle import attention
+
+    T, kb, vb = cfgd["T"], cfgd["k_bits"], cfgd["v_bits"]
+    heads, nbytes, spent = 0, 0.0, 0.0
+    while spent < seconds or heads == 0:
+        q, kg, vg = pool[heads % len(pool)]
+        t0 = time.perf_counter()
+        attention.decode_rotated(q, kg, vg)
+        spent += time.perf_counter() - t0
+        nbytes += T * packed_bytes_per_token_head(kb, vb, len(kg))
+        heads += 1
+    return nbytes / spent / 1e9, heads, spent
+
+
+def run_reference(args, rank, world):
+    from decode_attention_13_b200 import synth
+
+    cfgd = synth.CONFIGS[args.config]
+    if rank != 0:
+        return
+    pool = oracle_pool(cfgd)
+    threads = oracle_threads()
+    per_step = args.cpu_seconds / max(1, args.steps)
+    for _ in range(args.warmup):
+        oracle_decode_sample(cfgd, pool, 0.0)
+    vals, heads_total, spent_total = [], 0, 0.0
+    for _ in range(args.steps):
+        v, h, s = oracle_decode_sample(cfgd, pool, per_step)
+        vals.append(v)
+        heads_total += h
+        spent_total += s
+    value = statistics.mean(vals)
+    sample = ("oracle decode of %d whole KV heads (T=%d, G=%d query heads each) of the %s "
+              "workload; one bounded sample per step" % (heads_total, cfgd["T"],
+                                                         cfgd["h_q"] // cfgd["h_kv"], cfgd["name"]))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "ms_per_step": 1e3 * spent_total / max(1, args.steps), "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfgd["name"], "layers": cfgd["layers"], "batch": cfgd["B"],
+                   "q_heads": cfgd["h_q"], "kv_heads": cfgd["h_kv"], "seq_len": cfgd["T"],
+                   "k_bits": cfgd["k_bits"], "v_bits": cfgd["v_bits"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world):
+    import numpy as np
+    import torch
+
+    import decode_attention_13_b200 as gtq
+    from decode_attention_13_b200 import synth
+
+    cfgd = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    L, B, hq, hkv, T = cfgd["layers"], cfgd["B"], cfgd["h_q"], cfgd["h_kv"], cfgd["T"]
+    kb, vb, gq = cfgd["k_bits"], cfgd["v_bits"], cfgd["h_q"] // cfgd["h_kv"]
+    assert cfgd["dtype"] == "fp16"
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- build every layer's packed cache (energy, greedy, quantize-pack)
+    plans, packed, qs, outs, kv = [], [], [], [], []
+    for layer in range(L):
+        k, v, q = synth.layer_torch((args.config, rank, layer), B, hkv, gq, T,
+                                    theta=cfgd["theta"], decay=cfgd["decay"], device=dev)
+        cfg = gtq.make_config(B, hq, hkv, kb, vb, T)
+        with torch.cuda.stream(stream):
+            plan = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
+            buf = torch.empty(plan.packed_bytes, dtype=torch.uint8, device=dev)
+            gtq.gtq_quantize_pack(plan, k, v, 0, T, buf, stream=stream)
+        plans.append(plan)
+        packed.append(buf)
+        qs.append(q)
+        outs.append(torch.empty((B, hq, 128), dtype=torch.float32, device=dev))
+        kv.append((k, v))
+    stream.synchronize()
+    for p in plans:
+        rc = gtq.gtq_status(p)
+        if rc != gtq.GTQ_OK:
+            raise RuntimeError("status after quantize: " + gtq.strerror(rc))
+    g_k = []  # nonzero-width key groups of every head (norms read per token)
+    for p in plans:
+        bits = gtq.gtq_get_bits(p)
+        g_k.append([[len(set(int(x) for x in bits[b, h] if x > 0)) for h in range(hkv)]
+                    for b in range(B)])
+    bytes_per_layer = [sum(T * packed_bytes_per_token_head(kb, vb, g_k[l][b][h])
+                           for b in range(B) for h in range(hkv)) for l in range(L)]
+    step_bytes = float(sum(bytes_per_layer))
+
+    # ---- prefill timing: quantize-pack of every layer (A3-A6)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for layer in range(L):
+            k, v = kv[layer]
+            gtq.gtq_quantize_pack(plans[layer], k, v, 0, T, packed[layer], stream=stream)
+        ev1.record(stream)
+    stream.synchronize()
+    quant_ms = ev0.elapsed_time(ev1)
+    quant_bytes = float(L * B * hkv * T * 512) + step_bytes
+
+    # ---- the decode step, captured in a CUDA graph
+    def step():
+        for layer in range(L):
+            gtq.gtq_decode_attn(plans[layer], packed[layer], T, qs[layer], outs[layer],
+                                stream=stream)
+
+    for _ in range(2):
+        with torch.cuda.stream(stream):
+            step()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    stream.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # ---- per-call timing of gtq_decode_attn (roofline of the decode kernel)
+    call_ms = []
+    with torch.cuda.stream(stream):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(L)]
+        for _ in range(2):
+            for layer in range(L):
+                a, b = evs[layer]
+                a.record(stream)
+                gtq.gtq_decode_attn(plans[layer], packed[layer], T, qs[layer], outs[layer],
+                                    stream=stream)
+                b.record(stream)
+            stream.synchronize()
+            call_ms.append([a.elapsed_time(b) for a, b in evs])
+    per_call_ms = statistics.mean(call_ms[-1])
+    per_call_bytes = step_bytes / L
+
+    # ---- end to end through the ABI with host buffers
+    q_host = torch.stack(qs).cpu().pin_memory()
+    out_host = torch.empty((L, B, hq, 128), dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(q_host, device=dev)
+    out_dev = torch.empty((L, B, hq, 128), dtype=torch.float32, device=dev)
+
+    def e2e_step():
+        q_dev.copy_(q_host, non_blocking=True)
+        for layer in range(L):
+            gtq.gtq_decode_attn(plans[layer], packed[layer], T, q_dev[layer], out_dev[layer],
+                                stream=stream)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+    stream.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    ref_check = np.isfinite(out_host.numpy()).all()
+
+    # ---- CPU baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, heads, spent = oracle_decode_sample(cfgd, oracle_pool(cfgd), args.cpu_seconds)
+        threads = oracle_threads()
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "fp64 oracle decode of %d whole KV heads (T=%d, %d query heads "
+                         "each), %.1f s of CPU work" % (heads, T, gq, spent)}
+
+    hbm, peak_kind = peaks()
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    achieved = per_call_bytes / (per_call_ms * 1e-3) / 1e9
+    traffic = profile_traffic(os.path.join(ROOT, "decode_attention_13_b200", "csrc",
+                                           "gtq_decode.cu"))
+    n_launch = 3 * L * args.steps
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 operands / f32 accumulate", "data": "synthetic",
+        "config": {"workload": cfgd["name"], "layers": L, "batch": B, "q_heads": hq,
+                   "kv_heads": hkv, "seq_len": T, "k_bits": kb, "v_bits": vb,
+                   "parallelism": "replicas" if world == 1 else "dp%d (independent sequences)" % world,
+                   "l2": "cold: %.0f MB of packed cache per step > 126 MB L2, layers read in turn"
+                         % (step_bytes / 1e6)},
+        "pct_hbm_peak": 100.0 * value / world / hbm, "hbm_peak_gbs": hbm,
+        "pct_hbm_nominal_8tbs": 100.0 * value / world / 8000.0,
+        "ctx_tokens_per_s": world * B * T / (ms * 1e-3),
+        "bytes_per_step": step_bytes,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic,
+                     "kernel": "gtq_decode_attn call (rotate_q + decode_kernel + merge), "
+                               "CUDA events around each layer's call",
+                     "peak_kind": peak_kind},
+        "prefill": {"quantize_pack_ms_all_layers": quant_ms,
+                    "quantize_pack_gbs": quant_bytes / (quant_ms * 1e-3) / 1e9,
+                    "quantize_pack_frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / hbm},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
+                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+                "path": "pinned host q -> gtq_decode_attn per layer (eager) -> pinned host out; "
+                        "the packed cache stays resident"},
+        "gpu_launches": n_launch,
+        "clocks": clk,
+        "outputs_finite": bool(ref_check),
+    }
+    if cpu:
+        res["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    del graph
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch
+
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -176,7 +176,6 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
     }
     m.n_groups = ng;
     m.n_slots = slot;
-    m.n_ktiles = (slot + 7) / 8;
     // split rule: widest groups first until the unsplit rest holds <= 1/4 of the energy
     double tot = 0.0;
     for (int g = 0; g < ng; ++g) tot += gen[g];
@@ -188,24 +187,23 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
         rem -= gen[g];
       }
     }
-    int ns = 0;
-    for (int kt = 0; kt < 8; ++kt) {
-      m.kt_seg_start[kt] = (uint8_t)ns;
-      m.kt_seg_count[kt] = 0;
-      if (kt >= m.n_ktiles) continue;
-      for (int g = 0; g < ng; ++g) {
-        int a = m.grp_first_slot[g], e = a + grp_count[g];
-        int lo = max(a, 8 * kt), hi = min(e, 8 * kt + 8);
-        if (lo >= hi) continue;
-        m.seg_group[ns] = (uint8_t)g;
-        m.seg_lo[ns] = (uint8_t)(lo - 8 * kt);
-        m.seg_hi[ns] = (uint8_t)(hi - 8 * kt);
-        m.seg_last[ns] = (uint8_t)(e <= 8 * kt + 8);
-        ++ns;
-        ++m.kt_seg_count[kt];
+    // decode k-tiles: each group's slots in runs of at most 8 (one mma k-step of 16 coords)
+    int nk = 0;
+    for (int g = 0; g < ng; ++g) {
+      const int first = m.grp_first_slot[g], cnt = grp_count[g];
+      for (int off = 0; off < cnt; off += 8) {
+        m.kt_group[nk] = (uint8_t)g;
+        m.kt_first_slot[nk] = (uint8_t)(first + off);
+        m.kt_nslots[nk] = (uint8_t)min(8, cnt - off);
+        m.kt_flags[nk] = (uint8_t)((off == 0 ? 1 : 0) | (off + 8 >= cnt ? 2 : 0));
+        ++nk;
       }
     }
-    m.n_segs = ns;
+    for (int k = nk; k < kMaxKt; ++k) {
+      m.kt_group[k] = 0; m.kt_first_slot[k] = 0; m.kt_nslots[k] = 0; m.kt_flags[k] = 0;
+    }
+    m.n_ktiles = nk;
+    m.reserved = 0;
   }
   __syncthreads();
   // key rotation rows: M_h[pos][dim], pos = 2 * slot + e  <->  row r = 2 (slot - first) + e of R_m

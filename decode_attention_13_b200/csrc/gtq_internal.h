@@ -13,7 +13,7 @@ constexpr int kTile = GTQ_TILE_TOKENS;  // tokens per packed tile
 constexpr int kD = 128;                 // head_dim of quantize / decode
 constexpr int kBlocks = kD / 2;         // RoPE blocks per head
 constexpr int kMaxGroups = 8;           // one group per nonzero width 1..8
-constexpr int kMaxSegs = 16;            // (k-tile, group) intersections <= 8 + 8 - 1
+constexpr int kMaxKt = 16;              // group-pure decode k-tiles: <= 8 + (groups - 1)
 constexpr int kMaxGq = 8;               // query heads per KV head handled by decode
 constexpr int kLutEntries = 510;        // sum over w = 1..8 of 2^w
 constexpr int kThrEntries = 502;        // sum over w = 1..8 of (2^w - 1)
@@ -30,8 +30,8 @@ __host__ __device__ inline int thr_base(int w) { return (1 << w) - 1 - w; }
 struct HeadMeta {
   int32_t n_groups;  // G_K: nonzero-width groups
   int32_t n_slots;   // sum over groups of m/2
-  int32_t n_ktiles;  // ceil(n_slots / 8)
-  int32_t n_segs;    // (k-tile, group) segments
+  int32_t n_ktiles;  // decode k-tiles (16 coords each), every one inside one group
+  int32_t reserved;
   float inv_sqrt_m[kMaxGroups];
   float sqrt_m[kMaxGroups];
   uint8_t grp_width[kMaxGroups];  // descending
@@ -42,12 +42,10 @@ struct HeadMeta {
   uint8_t slot_group[kBlocks];
   uint16_t slot_koff[kBlocks];    // byte offset of the slot in the key-code area
   uint8_t block_group[kBlocks];   // group of each RoPE block (0xFF: width 0)
-  uint8_t kt_seg_start[8];
-  uint8_t kt_seg_count[8];
-  uint8_t seg_group[kMaxSegs];
-  uint8_t seg_lo[kMaxSegs];       // slot range [lo, hi) within the k-tile (0..8)
-  uint8_t seg_hi[kMaxSegs];
-  uint8_t seg_last[kMaxSegs];     // the group ends in this segment
+  uint8_t kt_group[kMaxKt];       // group of decode k-tile k
+  uint8_t kt_first_slot[kMaxKt];  // its slots: [first, first + n)
+  uint8_t kt_nslots[kMaxKt];      // 1..8
+  uint8_t kt_flags[kMaxKt];       // bit 0: first k-tile of its group, bit 1: last
 };
 
 // Device-resident constant tables shared by every plan of a (device, seed).
