@@ -44,6 +44,7 @@ ABI_FUNCTIONS = (
     "gtq_alloc_bits", "gtq_alloc_bits_from_energy", "gtq_quantize_pack", "gtq_decode_attn",
     "gtq_free", "gtq_packed_bytes", "gtq_get_bits", "gtq_get_energy", "gtq_status",
     "gtq_strerror", "gtq_last_error", "gtq_lloyd_max", "gtq_rotation", "gtq_layout_tile_bytes",
+    "gtq_block_energy_noalloc",
 )
 
 
@@ -95,6 +96,7 @@ def _load():
         "gtq_lloyd_max": (I32, [I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
         "gtq_rotation": (I32, [ctypes.c_uint64, I32, I32, ctypes.POINTER(ctypes.c_double)]),
         "gtq_layout_tile_bytes": (SZ, [I32, I32]),
+        "gtq_block_energy_noalloc": (I32, [ctypes.POINTER(gtq_config), P, I64, I64x4, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -10,6 +10,8 @@
 //   meta_kernel            groups (descending width), slots, decode segments and
 //                          the per-head key rotation rows M_h in packed order
 #include <cmath>
+#include <cstdio>
+#include <mutex>
 
 #include "gtq_internal.h"
 
@@ -262,3 +264,93 @@ cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s) {
 }
 
 }  // namespace gtq
+
+namespace gtq {
+
+// ---------------------------------------------------------------------------
+// Energy pass without any device allocation.
+//
+// gtq_alloc_bits gets its energy-pass scratch (fp64 partial sums per token
+// chunk) from cudaMallocAsync.  Some callers cannot allocate device memory at
+// call time: code that runs while a CUDA graph is being captured, servers that
+// reserve all device memory up front and forbid later allocations, and
+// real-time loops that cannot afford an allocator call.  gtq_block_energy_noalloc
+// runs the same two kernels with that scratch in the fixed array below instead.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocEnergyDoubles = (size_t)1 << 19;  // 4 MiB of partial sums per GPU
+
+// One copy per GPU that loads the library, alive until the process exits.
+static __device__ __align__(256) double g_energy_scratch[kNoAllocEnergyDoubles];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+double* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_energy_scratch on `device` (the current device); looked up
+// once per device.  In host code the array's name is only a host-side stand-in.
+cudaError_t scratch_for(int device, double** out) {
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_scratch_mu);
+  if (!g_scratch_ptr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_energy_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[device] = static_cast<double*>(p);
+  }
+  *out = g_scratch_ptr[device];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace gtq
+
+extern "C" int gtq_block_energy_noalloc(const gtq_config* cfg, const void* k_dev, int64_t T,
+                                        const int64_t k_strides[4], double* energy_dev,
+                                        void* stream) {
+  using namespace gtq;
+  if (!cfg || !k_dev || !k_strides || !energy_dev) return GTQ_ERR_INVALID;
+  if (cfg->batch < 1 || cfg->n_kv_heads < 1) return GTQ_ERR_INVALID;
+  if (cfg->head_dim < 8 || cfg->head_dim > kD || (cfg->head_dim % 8)) return GTQ_ERR_UNSUPPORTED;
+  if (cfg->rope_pairing != GTQ_PAIRING_HALF && cfg->rope_pairing != GTQ_PAIRING_INTERLEAVED)
+    return GTQ_ERR_INVALID;
+  if (cfg->in_dtype != GTQ_DTYPE_FP16 && cfg->in_dtype != GTQ_DTYPE_FP32) return GTQ_ERR_INVALID;
+  if (T < 1) return GTQ_ERR_INVALID;
+  const int esz = cfg->in_dtype == GTQ_DTYPE_FP16 ? 2 : 4;
+  if (k_strides[3] != 1 || ((uintptr_t)k_dev % 16) || ((uintptr_t)energy_dev % 8))
+    return GTQ_ERR_INVALID;
+  for (int i = 0; i < 3; ++i)
+    if (k_strides[i] < 0 || (k_strides[i] * esz) % 16) return GTQ_ERR_INVALID;
+  const int heads = cfg->batch * cfg->n_kv_heads;
+  const int64_t chunks = (T + kEnergyChunk - 1) / kEnergyChunk;
+  if ((double)heads * (double)chunks * 128.0 > (double)kNoAllocEnergyDoubles) {
+    char msg[160];
+    snprintf(msg, sizeof(msg),
+             "gtq_block_energy_noalloc: %d heads x %lld token chunks need %lld partial sums, "
+             "the fixed scratch holds %zu",
+             heads, (long long)chunks, (long long)heads * chunks * 128, kNoAllocEnergyDoubles);
+    set_last_error(msg);
+    return GTQ_ERR_UNSUPPORTED;
+  }
+  int device = 0;
+  double* part = nullptr;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e == cudaSuccess) e = scratch_for(device, &part);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  cudaStream_t s = (cudaStream_t)stream;
+  dim3 grid((unsigned)chunks, heads);
+  // every partial sum read by energy_finish_kernel is first written by
+  // energy_partial_kernel, so the shared scratch needs no clearing
+  if (cfg->in_dtype == GTQ_DTYPE_FP16)
+    energy_partial_kernel<__half><<<grid, 256, 0, s>>>((const __half*)k_dev, k_strides[0],
+                                                       k_strides[1], k_strides[2],
+                                                       cfg->n_kv_heads, cfg->head_dim, T, part);
+  else
+    energy_partial_kernel<float><<<grid, 256, 0, s>>>((const float*)k_dev, k_strides[0],
+                                                      k_strides[1], k_strides[2],
+                                                      cfg->n_kv_heads, cfg->head_dim, T, part);
+  energy_finish_kernel<<<heads, 64, 0, s>>>(part, (int)chunks, cfg->head_dim, cfg->rope_pairing,
+                                            T, energy_dev);
+  return record_cuda_error(cudaGetLastError());
+}

@@ -105,6 +105,11 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
 
 }  // namespace
 
+namespace gtq {
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+int record_cuda_error(cudaError_t e) { return cuda_code(e); }
+}  // namespace gtq
+
 extern "C" {
 
 size_t gtq_layout_tile_bytes(int32_t k_bits, int32_t v_bits) {

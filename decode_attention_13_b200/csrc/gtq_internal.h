@@ -90,6 +90,10 @@ struct gtq_plan {
 };
 
 namespace gtq {
+// Error text for gtq_last_error (gtq_api.cu)
+void set_last_error(const char* msg);
+int record_cuda_error(cudaError_t e);  // GTQ_OK, or GTQ_ERR_CUDA / GTQ_ERR_OOM with the text set
+
 // Host tables (gtq_tables.cu)
 int lloyd_max_host(int bits, double* c, double* t, double* d);
 int rotation_host(uint64_t seed, int tag, int m, double* out);

@@ -197,6 +197,34 @@ GTQ_API const char* gtq_strerror(int code);
  * into GTQ_ERR_CUDA / GTQ_ERR_OOM ("" if none); valid until the next call. */
 GTQ_API const char* gtq_last_error(void);
 
+/*
+ * gtq_block_energy_noalloc -- the energy pass of gtq_alloc_bits (E_i of every
+ * RoPE block of every (sequence, KV head), fp64, same kernels and summation
+ * order) without allocating any device memory.  The page has no counterpart:
+ * this entry point serves callers that cannot call cudaMalloc at call time --
+ * code running while a CUDA graph is captured, servers that reserve all
+ * device memory up front, real-time loops that cannot afford the allocator.
+ *   cfg         batch, n_kv_heads, head_dim (multiple of 8, <= 128),
+ *               rope_pairing and in_dtype are read; other fields are ignored.
+ *   k_dev       post-RoPE keys as in gtq_alloc_bits (same strides and alignment).
+ *   T           tokens to score, >= 1.
+ *   energy_dev  output, fp64 [batch][n_kv_heads][head_dim/2], 8-byte aligned,
+ *               caller-owned device memory, written in full.
+ * Scratch: a fixed 4 MiB array of partial sums inside the library (one per GPU
+ * that loads it, held until the process exits).  batch * n_kv_heads *
+ * ceil(T / 1024) * 128 must not exceed 2^19; larger calls return
+ * GTQ_ERR_UNSUPPORTED (gtq_last_error gives the sizes) and launch nothing.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array: calls that overlap on the GPU (different streams
+ * without ordering) race and give wrong energies.  Every scratch element a call
+ * reads it has written first, so no clearing is needed between calls.
+ * Errors: INVALID, UNSUPPORTED, CUDA.
+ */
+GTQ_API int gtq_block_energy_noalloc(const gtq_config* cfg, const void* k_dev, int64_t T,
+                                     const int64_t k_strides[4], double* energy_dev,
+                                     void* stream);
+
 /* Library's own tables, computed on the host (no GPU needed):
  * the b-bit Lloyd-Max quantizer of N(0,1) (b = 0..8): 2^b centroids
  * (ascending), 2^b - 1 thresholds and the distortion D(b). */
