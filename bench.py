@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's context length (overhead studies only)")
     return ap.parse_args()
 
 
@@ -208,7 +210,10 @@ def run_ours(args, rank, world):
     import decode_attention_13_b200 as gtq
     from decode_attention_13_b200 import synth
 
-    cfgd = synth.CONFIGS[args.config]
+    cfgd = dict(synth.CONFIGS[args.config])
+    if args.seq_len:
+        cfgd["T"] = args.seq_len
+        cfgd["name"] += " (context overridden to %d)" % args.seq_len
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     L, B, hq, hkv, T = cfgd["layers"], cfgd["B"], cfgd["h_q"], cfgd["h_kv"], cfgd["T"]

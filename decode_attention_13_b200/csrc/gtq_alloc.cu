@@ -191,8 +191,11 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
     }
     // decode k-tiles: each group's slots in runs of at most 8 (one mma k-step of 16 coords)
     int nk = 0;
+    for (int g = 0; g < kMaxGroups; ++g) m.grp_kt0[g] = m.grp_kt1[g] = 0;
     for (int g = 0; g < ng; ++g) {
       const int first = m.grp_first_slot[g], cnt = grp_count[g];
+      m.grp_kt0[g] = (uint8_t)nk;
+      m.grp_kt1[g] = (uint8_t)(nk + (cnt + 7) / 8);
       for (int off = 0; off < cnt; off += 8) {
         m.kt_group[nk] = (uint8_t)g;
         m.kt_first_slot[nk] = (uint8_t)(first + off);

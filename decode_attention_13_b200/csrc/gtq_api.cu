@@ -89,10 +89,10 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   alloc((void**)&p->d_meta, H * sizeof(HeadMeta));
   alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
   alloc((void**)&p->d_qrot, H * 8 * kD * sizeof(float));
-  alloc((void**)&p->d_partials, H * kMaxSplits * 8 * kPartialStride * sizeof(float));
-  alloc((void**)&p->d_tickets, H * sizeof(unsigned));
+  alloc((void**)&p->d_partials, H * kPartialSlots * 8 * kPartialStride * sizeof(float));
+  alloc((void**)&p->d_tickets, H * (1 + kMaxMergeGroups) * sizeof(unsigned));
   alloc((void**)&p->d_status, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * (1 + kMaxMergeGroups) * sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(p->d_meta, 0, H * sizeof(HeadMeta));
   if (e != cudaSuccess) {

@@ -19,6 +19,9 @@ constexpr int kLutEntries = 510;        // sum over w = 1..8 of 2^w
 constexpr int kThrEntries = 502;        // sum over w = 1..8 of (2^w - 1)
 constexpr int kMaxSplits = 256;         // context splits per head in decode
 constexpr int kPartialStride = 2 + kD;  // (m, l, o[128]) per (split, q head)
+constexpr int kMergeGroup = 16;          // splits merged together at the first merge level
+constexpr int kMaxMergeGroups = kMaxSplits / kMergeGroup;
+constexpr int kPartialSlots = kMaxSplits + kMaxMergeGroups;  // per head: level 1 + level 2
 constexpr int kStatusOverflow = 1;      // status word bits
 constexpr int kStatusTimeout = 2;
 
@@ -42,11 +45,25 @@ struct HeadMeta {
   uint8_t slot_group[kBlocks];
   uint16_t slot_koff[kBlocks];    // byte offset of the slot in the key-code area
   uint8_t block_group[kBlocks];   // group of each RoPE block (0xFF: width 0)
+  uint8_t grp_kt0[kMaxGroups];    // decode k-tiles of group g: [grp_kt0, grp_kt1)
+  uint8_t grp_kt1[kMaxGroups];
   uint8_t kt_group[kMaxKt];       // group of decode k-tile k
   uint8_t kt_first_slot[kMaxKt];  // its slots: [first, first + n)
   uint8_t kt_nslots[kMaxKt];      // 1..8
   uint8_t kt_flags[kMaxKt];       // bit 0: first k-tile of its group, bit 1: last
 };
+
+// Decode lookup tables, laid out exactly as the decode kernel's shared memory:
+// pair tables (widths 1..3, fp16 half2 (cb[c0], cb[c1]) at entry c0 | c1 << w,
+// one copy per lane: word offset kPairOff(w)/4 + entry * 32 + lane), then
+// single-code tables (widths 1..8, word kSingleOff(w)/4 + code = fp16 hi part in
+// the low half, fp16 lo part in the high half).  The offsets make
+// "offset | index" an address without an add.
+constexpr int kPairBytes = 10752;
+constexpr int kSingleBytes = 2048;
+constexpr int kDecodeImageBytes = kPairBytes + kSingleBytes;
+__host__ __device__ constexpr uint32_t kPairOff(int w) { return w == 3 ? 0u : (w == 2 ? 8192u : 10240u); }
+__host__ __device__ constexpr uint32_t kSingleOff(int w) { return 2048u - (8u << w); }
 
 // Device-resident constant tables shared by every plan of a (device, seed).
 struct Tables {
@@ -56,6 +73,7 @@ struct Tables {
   float* thr;        // fp32 thresholds, width w at thr_base(w)
   __half* lut_hi;    // fp16(centroid), width w at lut_base(w)
   __half* lut_lo;    // fp16(centroid - fp16(centroid))
+  uint4* dec_image;  // kDecodeImageBytes: the decode kernel's lookup tables
 };
 
 inline size_t rot_k_offset(int m) {  // element offset of R_m (m even) in rot_k
@@ -84,8 +102,8 @@ struct gtq_plan {
   gtq::HeadMeta* d_meta;  // [heads]
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
   float* d_qrot;      // [heads][8][128] rotated, scaled queries (decode workspace)
-  float* d_partials;  // [heads][kMaxSplits][8][kPartialStride]
-  unsigned* d_tickets;  // [heads]
+  float* d_partials;  // [heads][kPartialSlots][8][kPartialStride]
+  unsigned* d_tickets;  // [heads][1 + kMaxMergeGroups] arrival counters of the split merge
   int* d_status;      // device status word
 };
 
