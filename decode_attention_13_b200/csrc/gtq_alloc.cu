@@ -260,9 +260,13 @@ cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s) {
   greedy_kernel<<<(p->n_heads + warps - 1) / warps, 32 * warps, 0, s>>>(
       p->d_energy, p->tab.dist, p->n_blocks, p->cfg.k_bits, p->cfg.max_bits, p->n_heads,
       p->d_bits);
-  if (p->cfg.head_dim == kD)
+  if (p->cfg.head_dim == kD) {
     meta_kernel<<<p->n_heads, 128, 0, s>>>(p->d_bits, p->d_energy, p->tab.rot_k,
                                            p->cfg.rope_pairing, p->d_meta, p->d_mrow);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return build_b_images(p->d_mrow, p->n_heads, (size_t)kD * kD, p->d_bimg, s);
+  }
   return cudaGetLastError();
 }
 

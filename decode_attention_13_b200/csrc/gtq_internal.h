@@ -65,6 +65,21 @@ constexpr int kDecodeImageBytes = kPairBytes + kSingleBytes;
 __host__ __device__ constexpr uint32_t kPairOff(int w) { return w == 3 ? 0u : (w == 2 ? 8192u : 10240u); }
 __host__ __device__ constexpr uint32_t kSingleOff(int w) { return 2048u - (8u << w); }
 
+// Code lookup table of the tensor-core quantizer for widths 3..8: for |z| the
+// cell i = floor(|z| * inv[w]) (fp32 fma, round toward zero) holds at most one
+// positive threshold T (+inf if none) and the number of positive thresholds in
+// lower cells, so #{T_k < |z|} = base + (|z| > T).  Device blob: CodeLutMeta
+// (128 bytes) followed by float2 entries {T, base as int bits}.
+constexpr int kCodeLutEntries = 512;
+struct CodeLutMeta {
+  float inv[GTQ_MAX_BITS + 1];
+  int off[GTQ_MAX_BITS + 1];   // first entry of width w
+  int nmax[GTQ_MAX_BITS + 1];  // last cell of width w (no threshold, base = 2^(w-1) - 1)
+  int ok;                      // 1 when every cell holds at most one threshold
+};
+static_assert(sizeof(CodeLutMeta) <= 128, "code LUT header");
+constexpr size_t kCodeLutBytes = 128 + kCodeLutEntries * 8;
+
 // Device-resident constant tables shared by every plan of a (device, seed).
 struct Tables {
   double* rot_k;     // R_m for m = 2, 4, ..., 128, row-major, concatenated (fp64)
@@ -74,6 +89,8 @@ struct Tables {
   __half* lut_hi;    // fp16(centroid), width w at lut_base(w)
   __half* lut_lo;    // fp16(centroid - fp16(centroid))
   uint4* dec_image;  // kDecodeImageBytes: the decode kernel's lookup tables
+  uint8_t* rv_image; // R_V as the quantizer's tensor-core B operand (fp16 hi + lo, 64 KB)
+  uint8_t* code_lut; // kCodeLutBytes: CodeLutMeta + cells (built on the device from thr)
 };
 
 inline size_t rot_k_offset(int m) {  // element offset of R_m (m even) in rot_k
@@ -101,6 +118,7 @@ struct gtq_plan {
   uint8_t* d_bits;    // [heads][n_blocks]
   gtq::HeadMeta* d_meta;  // [heads]
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
+  uint8_t* d_bimg;    // [heads] M_h as the quantizer's tensor-core B operand (64 KB each)
   float* d_qrot;      // [heads][8][128] rotated, scaled queries (decode workspace)
   float* d_partials;  // [heads][kPartialSlots][8][kPartialStride]
   unsigned* d_tickets;  // [heads][1 + kMaxMergeGroups] arrival counters of the split merge
@@ -123,6 +141,14 @@ cudaError_t launch_energy(const gtq_plan* p, const void* k, int64_t T, const int
 cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s);
 cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
                             int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s);
+cudaError_t launch_quantize_cc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                               int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s);
+cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                               int64_t mt0, int64_t mt1, uint8_t* packed, cudaStream_t s);
+cudaError_t build_b_images(const float* rows, int count, size_t stride, uint8_t* img,
+                           cudaStream_t s);
+size_t b_image_bytes();
+cudaError_t build_code_lut(const float* thr, uint8_t* blob, cudaStream_t s);
 cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, const void* q,
                           int q_dtype, float* out, cudaStream_t s);
 }  // namespace gtq

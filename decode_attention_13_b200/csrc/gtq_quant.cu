@@ -270,8 +270,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
 
 }  // namespace
 
-cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                            int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s) {
+cudaError_t launch_quantize_cc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                               int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s) {
   QuantArgs a;
   a.k = k; a.v = v;
   a.s0 = st[0]; a.s1 = st[1]; a.s2 = st[2];
@@ -305,6 +305,26 @@ cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, con
     quantize_kernel<float><<<grid, kQThreads, smem, s>>>(a);
   }
   return cudaGetLastError();
+}
+
+// Whole 128-token tiles of fp16 inputs go to the tensor-core kernel; the ragged
+// edges (partial packed tiles, appends) and fp32 inputs to the CUDA-core kernel.
+cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                            int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s) {
+  if (p->cfg.in_dtype == GTQ_DTYPE_FP16 && p->cfg.head_dim == kD) {
+    const int64_t mt0 = (t0 + 127) / 128, mt1 = (t0 + n) / 128;
+    if (mt1 > mt0) {
+      cudaError_t e = launch_quantize_tc(p, k, v, st, mt0, mt1, packed, s);
+      if (e != cudaErrorNotSupported) {
+        if (e != cudaSuccess) return e;
+        if (mt0 * 128 > t0) e = launch_quantize_cc(p, k, v, st, t0, mt0 * 128 - t0, packed, s);
+        if (e == cudaSuccess && t0 + n > mt1 * 128)
+          e = launch_quantize_cc(p, k, v, st, mt1 * 128, t0 + n - mt1 * 128, packed, s);
+        return e;
+      }
+    }
+  }
+  return launch_quantize_cc(p, k, v, st, t0, n, packed, s);
 }
 
 }  // namespace gtq

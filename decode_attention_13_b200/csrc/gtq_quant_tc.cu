@@ -1,0 +1,826 @@
+// Tensor-core quantize-pack (fp16 K/V, head_dim 128): the per-token rotations
+// run as tcgen05 GEMMs with fp32 accumulators in tensor memory ("RoPE-Aware Bit
+// Allocation for KV-Cache Quantization", Abstract: Block-GTQ quantizes keys
+// "built on TurboQuant-MSE", whose coder rotates every normalised vector before
+// scalar Lloyd-Max coding).  Stored values are those of the CUDA-core quantizer
+// (gtq_quant.cu): per token and key group g, n = ||k_g||, code = number of fp32
+// thresholds below (sqrt(m)/n) (M_h k)_j, fp16(n) stored; values likewise with
+// one group of 128 and R_V.
+//
+// One launch; a CTA works on one head in one role (blockIdx.z: 0 keys, 1 values)
+// and walks 128-token tiles that lie inside the tokens being written.  Per tile:
+//   * code GEMM   D_c[coord][token] = R . X^T with R = M_h (keys) or R_V (values)
+//                 split into fp16 hi + lo parts (A operand, resident in shared
+//                 memory) and X the fp16 tile (B operand, TMA, 128B swizzle);
+//                 two tensor-memory accumulators of 128 columns.
+//   * gather GEMM D_p[token][row] = X . P^T with P a 0/1 matrix that lists the
+//                 dims of key group 0, then group 1, ... (each group padded to 8
+//                 rows); every output is one input element, so D_p holds the
+//                 exact fp16 inputs as fp32, grouped by key group.  For values P
+//                 is the identity.
+// Warps: 0 TMA producer; 1 tensor-memory owner and MMA issuer; 2-5 norm warps
+// (thread = token: group sums of squares from D_p); 6-13 code warps (thread =
+// rotated coordinate, 64 tokens: codes, bit packing in registers with one
+// partner lane, 8-byte stores straight into the packed tiles).
+//
+// Norms: the fp32 sum of exact squares has a rigorous relative error bound;
+// when fp16 rounding of every value inside the bound agrees, that is the stored
+// norm, otherwise (about 0.1-0.4 % of norms) the warp recomputes the sum in fp64
+// from the fp16 tile in shared memory.  Scales for the codes come from the same
+// norm (fp32 division).  Zero vectors get a NaN scale so that every code
+// comparison is false and the codes are 0.
+// Waits are bounded; on expiry the status word gets GTQ_ERR_TIMEOUT's bit.
+#include <cuda.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "gtq_internal.h"
+
+namespace gtq {
+namespace {
+
+constexpr int kTcWarps = 14;
+constexpr int kTcThreads = 32 * kTcWarps;
+constexpr int kMTile = 128;          // tokens per MMA tile (= 2 packed tiles)
+constexpr int kStages = 3;           // input tile stages
+constexpr uint64_t kTcWaitNs = 2000000000ull;  // bound of every barrier wait
+
+constexpr int kMaxPRows = 176;       // 128 dims + at most 6 padding rows for each of 8 groups
+constexpr int kMaxChunks = kMaxPRows / 8;
+constexpr int kScaleStride = 132;    // floats per (buffer, group) row of the scale table
+
+constexpr uint32_t kBBytes = 65536;      // R image: hi 32 KB, lo 32 KB
+constexpr uint32_t kStageBytes = 32768;  // X tile: 2 atoms x 128 rows x 128 B
+constexpr uint32_t kOffB = 0;
+constexpr uint32_t kOffP = kOffB + kBBytes;
+constexpr uint32_t kOffA = kOffP + kMaxPRows * 256;
+constexpr uint32_t kOffScale = kOffA + kStages * kStageBytes;                  // float [2][8][132]
+constexpr uint32_t kOffLut = kOffScale + 2 * kMaxGroups * kScaleStride * 4;  // code LUT blob
+constexpr uint32_t kOffThr = kOffLut + (uint32_t)kCodeLutBytes;               // float [4]
+constexpr uint32_t kOffMeta = kOffThr + 16;
+constexpr uint32_t kOffInfo = kOffMeta + ((sizeof(HeadMeta) + 15) & ~15);
+constexpr uint32_t kOffBar = kOffInfo + 512;
+constexpr int kNumBars = 17;
+constexpr uint32_t kTcSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(kOffP % 1024 == 0 && kOffA % 1024 == 0, "swizzled operands need 1024-byte alignment");
+static_assert(kTcSmem <= 232448, "shared memory budget");
+
+// barrier indices
+constexpr int kFull = 0;     // [3] X tile landed (TMA bytes)
+constexpr int kEmpty = 3;    // [3] X stage free: both GEMMs done + 4 norm warps
+constexpr int kPFull = 6;    // gather accumulator written
+constexpr int kPEmpty = 7;   // gather accumulator read by the 4 norm warps
+constexpr int kCFull = 8;    // [2] code accumulator written
+constexpr int kCEmpty = 10;  // [2] code accumulator read by the 8 code warps
+constexpr int kSFull = 12;   // [2] scales of a tile written by the 4 norm warps
+constexpr int kSEmpty = 14;  // [2] scales read by the 8 code warps
+constexpr int kRBar = 16;    // R image loaded
+
+// per-CTA gather layout (built once)
+struct GatherInfo {
+  int n_rows;      // P rows (multiple of 16)
+  int n_chunks;    // 8-row chunks that hold dims
+  int n_groups;
+  int pad;
+  uint8_t chunk_group[kMaxChunks];
+  uint8_t grp_row0[kMaxGroups];    // first P row of group g
+  uint8_t grp_rows[kMaxGroups];    // dims of group g (= m)
+  uint8_t grp_chunks[kMaxGroups];  // 8-row chunks of group g
+  float sqrt_m[kMaxGroups];
+  uint8_t row_dim[kMaxPRows];      // input dim of P row r (0xFF: padding)
+};
+static_assert(sizeof(GatherInfo) <= 512, "gather info");
+
+__host__ __device__ constexpr uint32_t idesc_f16(int n) {
+  // f32 accumulate, f16 A and B, both K-major, M = 128, N = n
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kMTile >> 4) << 24);
+}
+
+struct TcArgs {
+  const uint8_t* bimg_k;  // per head, kBBytes each
+  const uint8_t* bimg_v;  // one image
+  const HeadMeta* meta;
+  const float* thr;
+  const uint8_t* code_lut;
+  uint8_t* packed;
+  int64_t n_tiles;        // packed tiles per head (capacity)
+  int tile_bytes;
+  int kb, vb, pairing, hkv;
+  int64_t mt0, mt1;       // MMA tiles [mt0, mt1) of every head
+  int* status;
+};
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// bounded wait: gives up (returns false) after about two seconds
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = 0;
+  for (unsigned i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 255u) {
+      uint64_t now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t0 == 0)
+        t0 = now;
+      else if (now - t0 > kTcWaitNs)
+        return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// shared-memory matrix descriptor: K-major, 128B swizzle, 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) |
+         ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ void tc_mma(uint32_t tmem, uint64_t da, uint64_t db, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// What a code warp needs to turn scaled values into codes of width W.
+struct CodeCtx {
+  float t[3];           // widths 1-2: thresholds (width 1: t[0] = 0)
+  const float2* lut;    // widths 3-8: first cell of width W
+  float inv;            // cells per unit of |z|
+  uint32_t nmax;        // last cell
+};
+
+template <int W>
+__device__ __forceinline__ CodeCtx code_ctx(const float* thr4, const CodeLutMeta* lm,
+                                            const float2* cells) {
+  CodeCtx c;
+  if constexpr (W == 1) {
+    c.t[0] = thr4[0];
+  } else if constexpr (W == 2) {
+    c.t[0] = thr4[1]; c.t[1] = thr4[2]; c.t[2] = thr4[3];
+  } else {
+    c.lut = cells + lm->off[W];
+    c.inv = lm->inv[W];
+    c.nmax = (uint32_t)lm->nmax[W];
+  }
+  return c;
+}
+
+// Lloyd-Max code of z for width W: the number of thresholds t_i < z (a NaN z gives 0).
+// Widths 1-2 compare with thresholds in registers.  Wider ones use the symmetry of
+// the thresholds (the middle one is 0) and a uniform-cell table over |z|: the cell
+// of |z| holds at most one positive threshold T and the count of those below it,
+// so one load and one comparison give c = #{T_k < |z|} (z > 0: code H + c) or
+// c = #{T_k <= |z|} (code H - 1 - c); a NaN lands in the last cell (code 0).
+template <int W>
+__device__ __forceinline__ uint32_t lm_code(float z, const CodeCtx& c) {
+  if constexpr (W == 1) {
+    return z > c.t[0] ? 1u : 0u;
+  } else if constexpr (W == 2) {
+    return (z > c.t[0] ? 1u : 0u) + (z > c.t[1] ? 1u : 0u) + (z > c.t[2] ? 1u : 0u);
+  } else {
+    constexpr uint32_t H = 1u << (W - 1);
+    const float a = fabsf(z);
+    const uint32_t cell =
+        min(__float_as_uint(__fmaf_rz(a, c.inv, 8388608.f)) - 0x4B000000u, c.nmax);
+    const float2 e = c.lut[cell];
+    const bool pos = z > 0.f;
+    // z > 0: thresholds below z are the negative ones, 0 and the T_k < |z|;
+    // otherwise the negative thresholds -T_k < z, i.e. those with T_k > |z|
+    const uint32_t cnt = __float_as_uint(e.y) + ((pos ? a > e.x : a >= e.x) ? 1u : 0u);
+    return pos ? H + cnt : H - 1u - cnt;
+  }
+}
+
+// Bit of the lane's code for token jj (0..63) of a packed tile in the lane's
+// 4W-word stream, before the lane shift (keys: 8 portions (slot, g) of 16W bits,
+// code (u, e) at (2u + e)W with jj = g + 8u; values: 4 portions c of 32W bits,
+// code x at xW with x = 8b + 4k + 2h + l and jj = 16b + 8k + 2c + l).
+template <int ROLE, int W>
+__host__ __device__ constexpr int stream_bit(int jj) {
+  return ROLE == 0 ? 16 * W * (jj & 7) + 2 * W * (jj >> 3)
+                   : 32 * W * ((jj >> 1) & 3) + W * (8 * (jj >> 4) + 4 * ((jj >> 3) & 1) + (jj & 1));
+}
+
+// Codes of 32 tokens (half HALF of a packed tile) for the lane's coordinate, ORed
+// into the lane's stream.  y: accumulator columns, sc: the lane group's scales.
+template <int ROLE, int W, int HALF>
+__device__ __forceinline__ void code_half(const uint32_t (&y)[32], const float* sc,
+                                          const CodeCtx& ctx, uint32_t (&s)[32]) {
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sc + 4 * q4);
+    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int kk = 4 * q4 + i;
+      const uint32_t code = lm_code<W>(__uint_as_float(y[kk]) * sv[i], ctx);
+      const int bit = stream_bit<ROLE, W>(32 * HALF + kk);
+      s[bit >> 5] |= code << (bit & 31);
+      if ((bit & 31) + W > 32) s[(bit >> 5) + 1] |= code >> (32 - (bit & 31));
+    }
+  }
+}
+
+// The lane's fields sit e*W (keys) or 2h*W (values) bits further up; the partner
+// lane holds the other fields of the same portions.  Each lane keeps half of the
+// stream (keys: portions g = 4e..4e+3, values: c = 2h, 2h+1) and stores it: 8W bytes.
+template <int ROLE, int W>
+__device__ __forceinline__ void code_store(uint32_t (&s)[32], uint32_t side, unsigned mask,
+                                           uint8_t* dst) {
+  const uint32_t sh = ROLE == 0 ? side * W : side * 2 * W;
+#pragma unroll
+  for (int i = 4 * W - 1; i > 0; --i) s[i] = __funnelshift_l(s[i - 1], s[i], sh);
+  s[0] <<= sh;
+  uint32_t out[2 * W];
+#pragma unroll
+  for (int i = 0; i < 2 * W; ++i) {
+    const uint32_t send = side ? s[i] : s[2 * W + i];
+    const uint32_t recv = __shfl_xor_sync(mask, send, ROLE == 0 ? 1 : 8);
+    out[i] = (side ? s[2 * W + i] : s[i]) | recv;
+  }
+#pragma unroll
+  for (int i = 0; i < W; ++i)
+    *reinterpret_cast<uint2*>(dst + 8 * i) = make_uint2(out[2 * i], out[2 * i + 1]);
+}
+
+template <int ROLE, int HALF>
+__device__ __forceinline__ void code_half_w(int w, const uint32_t (&y)[32], const float* sc,
+                                            const float* thr4, const CodeLutMeta* lm,
+                                            const float2* cells, uint32_t (&s)[32]) {
+#define GTQ_CASE(W)                                                              \
+  case W:                                                                        \
+    code_half<ROLE, W, HALF>(y, sc, code_ctx<W>(thr4, lm, cells), s);            \
+    break;
+  switch (w) {
+    GTQ_CASE(1) GTQ_CASE(2) GTQ_CASE(3) GTQ_CASE(4)
+    GTQ_CASE(5) GTQ_CASE(6) GTQ_CASE(7) GTQ_CASE(8)
+    default: break;
+  }
+#undef GTQ_CASE
+}
+
+template <int ROLE>
+__device__ __forceinline__ void code_store_w(int w, uint32_t (&s)[32], uint32_t side,
+                                             unsigned mask, uint8_t* dst) {
+#define GTQ_CASE(W) case W: code_store<ROLE, W>(s, side, mask, dst); break;
+  switch (w) {
+    GTQ_CASE(1) GTQ_CASE(2) GTQ_CASE(3) GTQ_CASE(4)
+    GTQ_CASE(5) GTQ_CASE(6) GTQ_CASE(7) GTQ_CASE(8)
+    default: break;
+  }
+#undef GTQ_CASE
+}
+
+template <int ROLE>
+__device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = su32(sm);
+  const int head = blockIdx.y, bidx = head / a.hkv, hidx = head % a.hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* scale = reinterpret_cast<float*>(sm + kOffScale);
+  float* thr4 = reinterpret_cast<float*>(sm + kOffThr);
+  const CodeLutMeta* lut_meta = reinterpret_cast<const CodeLutMeta*>(sm + kOffLut);
+  const float2* lut_cells = reinterpret_cast<const float2*>(sm + kOffLut + 128);
+  HeadMeta& m = *reinterpret_cast<HeadMeta*>(sm + kOffMeta);
+  GatherInfo& gi = *reinterpret_cast<GatherInfo*>(sm + kOffInfo);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + kNumBars * 8);
+  const uint32_t bar0 = sb + kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar(kFull + i), 1);
+      mbar_init(bar(kEmpty + i), 1 + 4);
+    }
+    mbar_init(bar(kPFull), 1);
+    mbar_init(bar(kPEmpty), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kCFull + i), 1);
+      mbar_init(bar(kCEmpty + i), 8);
+      mbar_init(bar(kSFull + i), 4);
+      mbar_init(bar(kSEmpty + i), 8);
+    }
+    mbar_init(bar(kRBar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (tid < 4) thr4[tid] = a.thr[tid];  // width 1 (one threshold), width 2 (three)
+  for (int i = tid; i < (int)(kCodeLutBytes / 16); i += kTcThreads)
+    reinterpret_cast<uint4*>(sm + kOffLut)[i] = reinterpret_cast<const uint4*>(a.code_lut)[i];
+  if (ROLE == 0) {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(a.meta + head);
+    for (int i = tid; i < (int)(sizeof(HeadMeta) / 4); i += kTcThreads)
+      reinterpret_cast<uint32_t*>(&m)[i] = src[i];
+  }
+  __syncthreads();
+  if (tid == 0) {  // gather rows: the dims of every group in block order, groups padded to 8 rows
+    int row = 0, ch = 0;
+    const int ng = ROLE == 0 ? m.n_groups : 1;
+    for (int g = 0; g < ng; ++g) {
+      gi.grp_row0[g] = (uint8_t)row;
+      int cnt = 0;
+      if (ROLE == 0) {
+        for (int b = 0; b < kBlocks; ++b)
+          if (m.block_group[b] == g) {
+            gi.row_dim[row + cnt++] = (uint8_t)(a.pairing == GTQ_PAIRING_HALF ? b : 2 * b);
+            gi.row_dim[row + cnt++] = (uint8_t)(a.pairing == GTQ_PAIRING_HALF ? b + kBlocks : 2 * b + 1);
+          }
+        gi.sqrt_m[g] = m.sqrt_m[g];
+      } else {
+        for (int d = 0; d < kD; ++d) gi.row_dim[row + cnt++] = (uint8_t)d;
+        gi.sqrt_m[g] = 11.313708498984761f;  // sqrt(128)
+      }
+      gi.grp_rows[g] = (uint8_t)cnt;
+      const int nck = (cnt + 7) / 8;
+      gi.grp_chunks[g] = (uint8_t)nck;
+      for (int c = 0; c < nck; ++c) gi.chunk_group[ch + c] = (uint8_t)g;
+      for (int r = cnt; r < 8 * nck; ++r) gi.row_dim[row + r] = 0xFF;
+      row += 8 * nck;
+      ch += nck;
+    }
+    gi.n_chunks = ch;
+    gi.n_groups = ng;
+    gi.n_rows = row < 16 ? 16 : (row + 15) & ~15;
+    for (int r = row; r < gi.n_rows; ++r) gi.row_dim[r] = 0xFF;
+  }
+  __syncthreads();
+  const int n_rows = gi.n_rows;
+  if (ROLE == 0) {  // P image: zero, then one 1.0 per used row (keys only)
+    uint4* p = reinterpret_cast<uint4*>(sm + kOffP);
+    for (int i = tid; i < n_rows * 16; i += kTcThreads) p[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    for (int r = tid; r < n_rows; r += kTcThreads) {
+      const int d = gi.row_dim[r];
+      if (d != 0xFF)
+        *reinterpret_cast<uint16_t*>(sm + kOffP + (d >> 6) * (n_rows * 128) + r * 128 +
+                                     ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2) = 0x3C00;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+        su32(tmem_slot)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int64_t n_mt = a.mt1 - a.mt0;
+  int failed = 0;
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint8_t* rsrc = ROLE == 0 ? a.bimg_k + (size_t)head * kBBytes : a.bimg_v;
+      mbar_expect_tx(bar(kRBar), kBBytes);
+      bulk_load(sb + kOffB, rsrc, kBBytes, bar(kRBar));
+      int it = 0;
+      for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
+        const int st = it % kStages;
+        if (!mbar_wait(bar(kEmpty + st), ((it / kStages) & 1) ^ 1)) { failed = 1; break; }
+        const uint32_t dst = sb + kOffA + st * kStageBytes;
+        const int row = (int)((a.mt0 + t) * kMTile);
+        mbar_expect_tx(bar(kFull + st), kStageBytes);
+        tma_load_4d(dst, tmap, 0, row, hidx, bidx, bar(kFull + st));
+        tma_load_4d(dst + 16384, tmap, 64, row, hidx, bidx, bar(kFull + st));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      if (!mbar_wait(bar(kRBar), 0)) failed = 1;
+      const uint32_t idc = idesc_f16(kD), idp = idesc_f16(n_rows);
+      const uint32_t p_atom = (uint32_t)n_rows * 128;
+      int it = 0;
+      for (int64_t t = blockIdx.x; t < n_mt && !failed; t += gridDim.x, ++it) {
+        const int st = it % kStages, ac = it & 1;
+        if (!mbar_wait(bar(kFull + st), (it / kStages) & 1)) { failed = 1; break; }
+        const uint32_t x_base = sb + kOffA + st * kStageBytes;
+        if (ROLE == 0) {  // gather: D_p = X . P^T (key groups' dims, exact)
+          if (!mbar_wait(bar(kPEmpty), (it & 1) ^ 1)) { failed = 1; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc_mma(tmem + 256, smem_desc(x_base + (ks >> 2) * 16384 + (ks & 3) * 32),
+                   smem_desc(sb + kOffP + (ks >> 2) * p_atom + (ks & 3) * 32), idp, ks != 0);
+          tc_commit(bar(kPFull));
+        }
+        if (!mbar_wait(bar(kCEmpty + ac), ((it >> 1) & 1) ^ 1)) { failed = 1; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {  // code: D_c = (R_hi + R_lo) . X^T
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+            tc_mma(tmem + (uint32_t)(ac * kD), smem_desc(sb + kOffB + part * 32768 + koff),
+                   smem_desc(x_base + koff), idc, (part | ks) != 0);
+          }
+        }
+        tc_commit(bar(kCFull + ac));
+        tc_commit(bar(kEmpty + st));
+      }
+    }
+  } else if (warp < 6) {
+    // ----------------------------------------------------------- norm warps
+    const int q = warp & 3, j = 32 * q + lane;  // token of the tile (= tensor-memory lane)
+    const uint32_t trow = tmem + 256 + ((uint32_t)(32 * q) << 16);
+    const int norm_off = ROLE == 0 ? 1024 * (a.kb + a.vb) + 128 : 1024 * (a.kb + a.vb);
+    const int jj = j & 63, npos = 2 * ((jj & 7) * 8 + (jj >> 3));
+    const int n_chunks = gi.n_chunks;
+    int ovf = 0, it = 0;
+    for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
+      const int st = it % kStages, par = it & 1;
+      if (ROLE == 0) {
+        if (!mbar_wait(bar(kPFull), it & 1)) { failed = 1; break; }
+      } else {
+        if (!mbar_wait(bar(kFull + st), (it / kStages) & 1)) { failed = 1; break; }
+      }
+      if (!mbar_wait(bar(kSEmpty + par), ((it >> 1) & 1) ^ 1)) { failed = 1; break; }
+      tc_fence_after();
+      uint8_t* tile_base =
+          a.packed + ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + (j >> 6))) * a.tile_bytes;
+      const uint8_t* xt = sm + kOffA + st * kStageBytes;
+      float* sc_par = scale + par * kMaxGroups * kScaleStride;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      // one group is complete: stored norm and scale of token j
+      auto finish = [&](int g) {
+        const float S = (a0 + a1) + (a2 + a3);
+        float r;
+        asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(S));
+        const float n = S * r;
+        // relative error of n: at most (chunks + 1) roundings of the sum's 2^-24
+        // (halved by the root), the approximate reciprocal root and one product
+        const float delta = (float)(gi.grp_chunks[g] + 12) * 5.9604645e-8f;
+        const float lo = n * (1.f - delta), hi = n * (1.f + delta);
+        __half h = __ushort_as_half(0);
+        float sv = __int_as_float(0x7fc00000);  // NaN: zero vector, codes 0
+        bool amb = false;
+        if (S == 0.f) {
+        } else if (lo > 65504.f) {
+          h = __ushort_as_half(0x7BFF);
+          ovf = 1;
+          sv = gi.sqrt_m[g] * r;
+        } else if (hi <= 65504.f &&
+                   __half_as_ushort(__float2half_rn(lo)) == __half_as_ushort(__float2half_rn(hi))) {
+          h = __float2half_rn(n);
+          sv = gi.sqrt_m[g] * r;
+        } else {
+          amb = true;
+        }
+        unsigned am = __ballot_sync(0xffffffffu, amb);
+        while (am) {  // fp64 sum of the exact squares for one token, the whole warp helping
+          const int src = __ffs(am) - 1;
+          am &= am - 1;
+          const int jt = 32 * q + src;
+          double acc = 0.0;
+          for (int rr = lane; rr < gi.grp_rows[g]; rr += 32) {
+            const int d = gi.row_dim[gi.grp_row0[g] + rr];
+            const __half x = *reinterpret_cast<const __half*>(
+                xt + (d >> 6) * 16384 + jt * 128 + ((((d >> 3) & 7) ^ (jt & 7)) << 4) + (d & 7) * 2);
+            const double xd = (double)__half2float(x);
+            acc = fma(xd, xd, acc);
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == src) {
+            const double n64 = sqrt(acc);
+            if (n64 > 65504.0) ovf = 1;
+            h = __double2half(n64 > 65504.0 ? 65504.0 : n64);
+            sv = (float)((double)gi.sqrt_m[g] / n64);
+          }
+        }
+        *reinterpret_cast<__half*>(tile_base + norm_off + g * 128 + npos) = h;
+        sc_par[g * kScaleStride + j] = sv;
+      };
+      if (ROLE == 0) {
+        // group sums of squares from the gathered exact inputs, 8 columns per chunk
+        int cur = 0;
+        for (int b = 0; b < n_chunks; b += 4) {
+          uint32_t r[32];
+          tc_ld32(trow + 8 * b, r);
+          tc_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (b + k < n_chunks) {
+              const int g = gi.chunk_group[b + k];
+              if (g != cur) {
+                finish(cur);
+                a0 = a1 = a2 = a3 = 0.f;
+                cur = g;
+              }
+#pragma unroll
+              for (int e = 0; e < 8; e += 4) {
+                const float x0 = __uint_as_float(r[8 * k + e]), x1 = __uint_as_float(r[8 * k + e + 1]);
+                const float x2 = __uint_as_float(r[8 * k + e + 2]), x3 = __uint_as_float(r[8 * k + e + 3]);
+                a0 = fmaf(x0, x0, a0); a1 = fmaf(x1, x1, a1); a2 = fmaf(x2, x2, a2); a3 = fmaf(x3, x3, a3);
+              }
+            }
+          }
+        }
+        if (gi.n_groups > 0) finish(cur);
+      } else {
+        // values: one group of all 128 dims, straight from the fp16 tile (row j, 16-byte
+        // chunk c at position c ^ (j % 8) of its 128-byte row)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              xt + (c >> 3) * 16384 + j * 128 + ((uint32_t)((c & 7) ^ (j & 7)) << 4));
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&v.z));
+          const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&v.w));
+          a0 = fmaf(f0.x, f0.x, a0); a1 = fmaf(f0.y, f0.y, a1);
+          a2 = fmaf(f1.x, f1.x, a2); a3 = fmaf(f1.y, f1.y, a3);
+          a0 = fmaf(f2.x, f2.x, a0); a1 = fmaf(f2.y, f2.y, a1);
+          a2 = fmaf(f3.x, f3.x, a2); a3 = fmaf(f3.y, f3.y, a3);
+        }
+        finish(0);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (ROLE == 0) mbar_arrive(bar(kPEmpty));
+        mbar_arrive(bar(kEmpty + st));
+        mbar_arrive(bar(kSFull + par));
+      }
+    }
+    if (ovf) atomicOr(a.status, kStatusOverflow);
+  } else {
+    // ----------------------------------------------------------- code warps
+    const int q = warp & 3, hc = (warp - 6) >> 2;
+    const int c = 32 * q + lane;  // rotated coordinate = tensor-memory lane
+    int w, grp;
+    uint32_t side;
+    int dst_off;
+    if (ROLE == 0) {
+      const int slot = c >> 1;
+      w = slot < m.n_slots ? m.slot_width[slot] : 0;
+      grp = slot < m.n_slots ? m.slot_group[slot] : 0;
+      side = (uint32_t)(c & 1);
+      dst_off = slot < m.n_slots ? m.slot_koff[slot] + 8 * w * (c & 1) : 0;
+    } else {
+      w = a.vb;
+      grp = 0;
+      side = (uint32_t)((c >> 3) & 1);
+      dst_off = 1024 * a.kb + 16 * a.vb * (8 * (c >> 4) + (c & 7)) + 8 * a.vb * (int)side;
+    }
+    const unsigned mask = __match_any_sync(0xffffffffu, w);
+    const uint32_t tcol = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * hc);
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
+      const int ac = it & 1, par = it & 1;
+      if (!mbar_wait(bar(kSFull + par), (it >> 1) & 1)) { failed = 1; break; }
+      if (!mbar_wait(bar(kCFull + ac), (it >> 1) & 1)) { failed = 1; break; }
+      tc_fence_after();
+      const float* sc = scale + (par * kMaxGroups + grp) * kScaleStride + 64 * hc;
+      uint32_t s[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = 0;
+      {
+        uint32_t y[32];
+        tc_ld32(tcol + (uint32_t)(ac * kD), y);
+        tc_wait_ld();
+        code_half_w<ROLE, 0>(w, y, sc, thr4, lut_meta, lut_cells, s);
+      }
+      {
+        uint32_t y[32];
+        tc_ld32(tcol + (uint32_t)(ac * kD) + 32, y);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kCEmpty + ac));  // accumulator may be overwritten
+        code_half_w<ROLE, 1>(w, y, sc + 32, thr4, lut_meta, lut_cells, s);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kSEmpty + par));  // scales read
+      uint8_t* dst = a.packed +
+                     ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + hc)) * a.tile_bytes +
+                     dst_off;
+      code_store_w<ROLE>(w, s, side, mask, dst);
+    }
+  }
+  if (failed) atomicOr(a.status, kStatusTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, TcArgs a) {
+  if (blockIdx.z == 0)
+    tc_role<0>(&tmk, a);
+  else
+    tc_role<1>(&tmv, a);
+}
+
+// R image of a 128 x 128 matrix (rows = output coordinate, cols = input dim):
+// fp16 hi part then fp16 lo part, each K-major with the 128B swizzle.
+__global__ void b_image_kernel(const float* __restrict__ rows, size_t row_stride_heads,
+                               uint8_t* __restrict__ img) {
+  const float* r = rows + (size_t)blockIdx.x * row_stride_heads;
+  uint8_t* o = img + (size_t)blockIdx.x * kBBytes;
+  for (int i = threadIdx.x; i < kD * kD; i += blockDim.x) {
+    const int n = i / kD, d = i % kD;
+    const float v = r[i];
+    const __half hi = __float2half_rn(v);
+    const __half lo = __float2half_rn(v - __half2float(hi));
+    const uint32_t off = (d >> 6) * 16384 + n * 128 + ((((d >> 3) & 7) ^ (n & 7)) << 4) + (d & 7) * 2;
+    *reinterpret_cast<__half*>(o + off) = hi;
+    *reinterpret_cast<__half*>(o + 32768 + off) = lo;
+  }
+}
+
+// Cell of |z| in the code table: floor(|z| * inv) as an fp32 fma rounded toward
+// zero onto 2^23 (the same expression the quantizer evaluates).
+__device__ __forceinline__ uint32_t code_cell(float a, float inv) {
+  return __float_as_uint(__fmaf_rz(a, inv, 8388608.f)) - 0x4B000000u;
+}
+
+// Builds the code table of widths 3..8 from the fp32 thresholds (one thread).
+__global__ void code_lut_kernel(const float* __restrict__ thr, uint8_t* __restrict__ blob) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  CodeLutMeta* lm = reinterpret_cast<CodeLutMeta*>(blob);
+  float2* cells = reinterpret_cast<float2*>(blob + 128);
+  for (int w = 0; w <= GTQ_MAX_BITS; ++w) {
+    lm->inv[w] = 0.f;
+    lm->off[w] = 0;
+    lm->nmax[w] = 0;
+  }
+  int off = 0, ok = 1;
+  for (int w = 3; w <= GTQ_MAX_BITS && ok; ++w) {
+    const float* t = thr + thr_base(w);
+    const int H = 1 << (w - 1);  // t[H - 1] = 0; positive thresholds t[H .. 2H - 2]
+    float gap = INFINITY;
+    for (int k = H; k <= 2 * H - 2; ++k) gap = fminf(gap, t[k] - t[k - 1]);
+    const float inv = 1.f / (0.98f * gap);
+    const int n = (int)code_cell(t[2 * H - 2], inv) + 2;  // the last cell holds no threshold
+    if (off + n > kCodeLutEntries) {
+      ok = 0;
+      break;
+    }
+    for (int i = 0; i < n; ++i) cells[off + i] = make_float2(INFINITY, __int_as_float(0));
+    for (int k = H; k <= 2 * H - 2; ++k) {
+      const uint32_t c = code_cell(t[k], inv);
+      if (cells[off + c].x != INFINITY) ok = 0;
+      cells[off + c].x = t[k];
+    }
+    int below = 0, k = H;
+    for (int i = 0; i < n; ++i) {
+      while (k <= 2 * H - 2 && (int)code_cell(t[k], inv) < i) {
+        ++below;
+        ++k;
+      }
+      cells[off + i].y = __int_as_float(below);
+    }
+    lm->inv[w] = inv;
+    lm->off[w] = off;
+    lm->nmax[w] = n - 1;
+    off += n;
+  }
+  lm->ok = ok;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t build_b_images(const float* rows, int count, size_t stride, uint8_t* img,
+                           cudaStream_t s) {
+  b_image_kernel<<<count, 256, 0, s>>>(rows, stride, img);
+  return cudaGetLastError();
+}
+
+size_t b_image_bytes() { return kBBytes; }
+
+cudaError_t build_code_lut(const float* thr, uint8_t* blob, cudaStream_t s) {
+  code_lut_kernel<<<1, 32, 0, s>>>(thr, blob);
+  return cudaGetLastError();
+}
+
+// Quantize MMA tiles [mt0, mt1) of every head (keys and values in one launch).
+// Returns cudaErrorNotSupported when the inputs cannot be described by a tensor map.
+cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                               int64_t mt0, int64_t mt1, uint8_t* packed, cudaStream_t s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap maps[2];
+  const void* src[2] = {k, v};
+  for (int r = 0; r < 2; ++r) {
+    if (((uintptr_t)src[r] & 15) || ((st[0] * 2) & 15) || ((st[1] * 2) & 15) || ((st[2] * 2) & 15))
+      return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)(mt1 * kMTile),
+                                (cuuint64_t)p->cfg.n_kv_heads, (cuuint64_t)p->cfg.batch};
+    const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2,
+                                   (cuuint64_t)st[0] * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kMTile, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(&maps[r], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(src[r]), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  TcArgs a;
+  a.bimg_k = p->d_bimg;
+  a.bimg_v = p->tab.rv_image;
+  a.meta = p->d_meta;
+  a.thr = p->tab.thr;
+  a.code_lut = p->tab.code_lut;
+  a.packed = packed;
+  a.n_tiles = p->n_tiles;
+  a.tile_bytes = (int)p->tile_bytes;
+  a.kb = p->cfg.k_bits;
+  a.vb = p->cfg.v_bits;
+  a.pairing = p->cfg.rope_pairing;
+  a.hkv = p->cfg.n_kv_heads;
+  a.mt0 = mt0;
+  a.mt1 = mt1;
+  a.status = p->d_status;
+  const int64_t n_mt = mt1 - mt0;
+  const int per_head =
+      (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, p->n_sms / std::max(1, 2 * p->n_heads)));
+  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+  if (e != cudaSuccess) return e;
+  quantize_tc_kernel<<<dim3(per_head, p->n_heads, 2), kTcThreads, kTcSmem, s>>>(maps[0], maps[1], a);
+  return cudaGetLastError();
+}
+
+}  // namespace gtq

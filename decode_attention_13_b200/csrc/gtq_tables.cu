@@ -278,6 +278,20 @@ int tables_for(int device, uint64_t seed, Tables* out) {
   if (e == cudaSuccess) e = up((void**)&t.lut_hi, lhi.data(), lhi.size() * sizeof(__half));
   if (e == cudaSuccess) e = up((void**)&t.lut_lo, llo.data(), llo.size() * sizeof(__half));
   if (e == cudaSuccess) e = up((void**)&t.dec_image, img.data(), img.size() * sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMalloc((void**)&t.rv_image, b_image_bytes());
+  if (e == cudaSuccess) e = build_b_images(t.rot_v, 1, 0, t.rv_image, 0);
+  if (e == cudaSuccess) e = cudaMalloc((void**)&t.code_lut, kCodeLutBytes);
+  if (e == cudaSuccess) e = build_code_lut(t.thr, t.code_lut, 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) {
+    CodeLutMeta lm;
+    e = cudaMemcpy(&lm, t.code_lut, sizeof(lm), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && lm.ok != 1) {
+      cudaSetDevice(prev);
+      set_last_error("code lookup table: two thresholds share a cell");
+      return GTQ_ERR_CUDA;
+    }
+  }
   cudaSetDevice(prev);
   if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? GTQ_ERR_OOM : GTQ_ERR_CUDA;
   cache[key] = t;
