@@ -65,20 +65,25 @@ constexpr int kDecodeImageBytes = kPairBytes + kSingleBytes;
 __host__ __device__ constexpr uint32_t kPairOff(int w) { return w == 3 ? 0u : (w == 2 ? 8192u : 10240u); }
 __host__ __device__ constexpr uint32_t kSingleOff(int w) { return 2048u - (8u << w); }
 
-// Code lookup table of the tensor-core quantizer for widths 3..8: for |z| the
-// cell i = floor(|z| * inv[w]) (fp32 fma, round toward zero) holds at most one
-// positive threshold T (+inf if none) and the number of positive thresholds in
-// lower cells, so #{T_k < |z|} = base + (|z| > T).  Device blob: CodeLutMeta
-// (128 bytes) followed by float2 entries {T, base as int bits}.
-constexpr int kCodeLutEntries = 512;
+// Code lookup table of the tensor-core quantizer, one part per width w = 1..8.
+// Cell of an fp32 value z: floor(z * inv[w]) + k[w], evaluated as
+// fma(z, inv, 2^23 + k) rounded toward zero (the result's bits minus those of
+// 2^23), clamped to [0, nmax].  The function is monotone, every cell holds at
+// most one threshold T of width w (+inf if none), and the entry keeps T and the
+// number of thresholds in lower cells, so the code #{t_i < z} = base + (z > T).
+// Cell 0 and cell nmax hold no threshold.  Device blob: CodeLutMeta (kCodeLutHeader
+// bytes) followed by float2 entries {T, base as int bits}.
+constexpr int kCodeLutEntries = 1024;
 struct CodeLutMeta {
   float inv[GTQ_MAX_BITS + 1];
-  int off[GTQ_MAX_BITS + 1];   // first entry of width w
-  int nmax[GTQ_MAX_BITS + 1];  // last cell of width w (no threshold, base = 2^(w-1) - 1)
-  int ok;                      // 1 when every cell holds at most one threshold
+  float cadd[GTQ_MAX_BITS + 1];  // 2^23 + k[w]
+  int off[GTQ_MAX_BITS + 1];     // first entry of width w
+  int nmax[GTQ_MAX_BITS + 1];    // last cell of width w
 };
-static_assert(sizeof(CodeLutMeta) <= 128, "code LUT header");
-constexpr size_t kCodeLutBytes = 128 + kCodeLutEntries * 8;
+constexpr int kCodeLutHeader = 256;
+static_assert(sizeof(CodeLutMeta) <= kCodeLutHeader - 4, "code LUT header");
+constexpr int kCodeLutOkOffset = kCodeLutHeader - 4;  // int: 1 when the table is valid
+constexpr size_t kCodeLutBytes = kCodeLutHeader + kCodeLutEntries * 8;
 
 // Device-resident constant tables shared by every plan of a (device, seed).
 struct Tables {

@@ -57,8 +57,8 @@ constexpr uint32_t kOffP = kOffB + kBBytes;
 constexpr uint32_t kOffA = kOffP + kMaxPRows * 256;
 constexpr uint32_t kOffScale = kOffA + kStages * kStageBytes;                  // float [2][8][132]
 constexpr uint32_t kOffLut = kOffScale + 2 * kMaxGroups * kScaleStride * 4;  // code LUT blob
-constexpr uint32_t kOffThr = kOffLut + (uint32_t)kCodeLutBytes;               // float [4]
-constexpr uint32_t kOffMeta = kOffThr + 16;
+constexpr uint32_t kOffFlags = kOffLut + (uint32_t)kCodeLutBytes;  // uint8 [2][4] zero-norm flags
+constexpr uint32_t kOffMeta = kOffFlags + 16;
 constexpr uint32_t kOffInfo = kOffMeta + ((sizeof(HeadMeta) + 15) & ~15);
 constexpr uint32_t kOffBar = kOffInfo + 512;
 constexpr int kNumBars = 17;
@@ -200,134 +200,120 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// What a code warp needs to turn scaled values into codes of width W.
-struct CodeCtx {
-  float t[3];           // widths 1-2: thresholds (width 1: t[0] = 0)
-  const float2* lut;    // widths 3-8: first cell of width W
-  float inv;            // cells per unit of |z|
-  uint32_t nmax;        // last cell
+// Per-lane constants of the code stage (the lane's coordinate has width w).
+struct CodeLane {
+  float inv, cadd;      // cell function of width w
+  uint32_t lut_base;    // shared address of width w's entries minus 8 * bits(2^23)
+  int lo, hi;           // clamp of the raw cell bits: bits(2^23) + [0, nmax]
+  uint32_t sel_even, sel_odd;  // byte selectors of the merge with the partner lane
+  uint32_t mA, mB, m2;  // byte pairs (1, 2^w) at bytes 0-1 / 2-3 and 2^(2w) for compressing
+  uint32_t s4;          // 4w
+  int w;
 };
 
-template <int W>
-__device__ __forceinline__ CodeCtx code_ctx(const float* thr4, const CodeLutMeta* lm,
-                                            const float2* cells) {
-  CodeCtx c;
-  if constexpr (W == 1) {
-    c.t[0] = thr4[0];
-  } else if constexpr (W == 2) {
-    c.t[0] = thr4[1]; c.t[1] = thr4[2]; c.t[2] = thr4[3];
-  } else {
-    c.lut = cells + lm->off[W];
-    c.inv = lm->inv[W];
-    c.nmax = (uint32_t)lm->nmax[W];
-  }
-  return c;
+// Code of z: the number of thresholds t_i < z, from the cell table (one load,
+// one comparison; exact because cells are monotone and hold one threshold).
+__device__ __forceinline__ uint32_t code_of(float z, const CodeLane& L) {
+  int b = __float_as_int(__fmaf_rz(z, L.inv, L.cadd));
+  b = min(max(b, L.lo), L.hi);
+  uint32_t tb, base;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(tb), "=r"(base) : "r"(L.lut_base + ((uint32_t)b << 3)));
+  return base + (z > __uint_as_float(tb) ? 1u : 0u);
 }
 
-// Lloyd-Max code of z for width W: the number of thresholds t_i < z (a NaN z gives 0).
-// Widths 1-2 compare with thresholds in registers.  Wider ones use the symmetry of
-// the thresholds (the middle one is 0) and a uniform-cell table over |z|: the cell
-// of |z| holds at most one positive threshold T and the count of those below it,
-// so one load and one comparison give c = #{T_k < |z|} (z > 0: code H + c) or
-// c = #{T_k <= |z|} (code H - 1 - c); a NaN lands in the last cell (code 0).
-template <int W>
-__device__ __forceinline__ uint32_t lm_code(float z, const CodeCtx& c) {
-  if constexpr (W == 1) {
-    return z > c.t[0] ? 1u : 0u;
-  } else if constexpr (W == 2) {
-    return (z > c.t[0] ? 1u : 0u) + (z > c.t[1] ? 1u : 0u) + (z > c.t[2] ? 1u : 0u);
-  } else {
-    constexpr uint32_t H = 1u << (W - 1);
-    const float a = fabsf(z);
-    const uint32_t cell =
-        min(__float_as_uint(__fmaf_rz(a, c.inv, 8388608.f)) - 0x4B000000u, c.nmax);
-    const float2 e = c.lut[cell];
-    const bool pos = z > 0.f;
-    // z > 0: thresholds below z are the negative ones, 0 and the T_k < |z|;
-    // otherwise the negative thresholds -T_k < z, i.e. those with T_k > |z|
-    const uint32_t cnt = __float_as_uint(e.y) + ((pos ? a > e.x : a >= e.x) ? 1u : 0u);
-    return pos ? H + cnt : H - 1u - cnt;
-  }
+// Byte of the lane's code for token jj (0..63) of a packed tile: word jj_word,
+// byte jj_byte of 16 words.  Keys: portion g = jj % 8 (8 codes u = jj / 8) in
+// words 2g, 2g + 1.  Values: portion c = (jj / 2) % 4, own index 4b + 2k + l with
+// jj = 16b + 8k + 2c + l, in words 4c + b.  Either way the lane with side s keeps
+// words 8s..8s+7 (4 key portions g = 4s..4s+3 / 2 value portions c = 2s, 2s+1).
+template <int ROLE>
+__host__ __device__ constexpr int code_word(int jj) {
+  return ROLE == 0 ? 2 * (jj & 7) + (jj >> 5) : 4 * ((jj >> 1) & 3) + (jj >> 4);
+}
+template <int ROLE>
+__host__ __device__ constexpr int code_byte(int jj) {
+  return ROLE == 0 ? (jj >> 3) & 3 : 2 * ((jj >> 3) & 1) + (jj & 1);
 }
 
-// Bit of the lane's code for token jj (0..63) of a packed tile in the lane's
-// 4W-word stream, before the lane shift (keys: 8 portions (slot, g) of 16W bits,
-// code (u, e) at (2u + e)W with jj = g + 8u; values: 4 portions c of 32W bits,
-// code x at xW with x = 8b + 4k + 2h + l and jj = 16b + 8k + 2c + l).
-template <int ROLE, int W>
-__host__ __device__ constexpr int stream_bit(int jj) {
-  return ROLE == 0 ? 16 * W * (jj & 7) + 2 * W * (jj >> 3)
-                   : 32 * W * ((jj >> 1) & 3) + W * (8 * (jj >> 4) + 4 * ((jj >> 3) & 1) + (jj & 1));
-}
-
-// Codes of 32 tokens (half HALF of a packed tile) for the lane's coordinate, ORed
-// into the lane's stream.  y: accumulator columns, sc: the lane group's scales.
-template <int ROLE, int W, int HALF>
+// Codes of 32 tokens (half HALF of the packed tile) into the lane's byte words.
+template <int ROLE, int HALF, bool ZMASK>
 __device__ __forceinline__ void code_half(const uint32_t (&y)[32], const float* sc,
-                                          const CodeCtx& ctx, uint32_t (&s)[32]) {
+                                          const CodeLane& L, uint32_t (&A)[16]) {
 #pragma unroll
   for (int q4 = 0; q4 < 8; ++q4) {
     const float4 s4 = *reinterpret_cast<const float4*>(sc + 4 * q4);
     const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int kk = 4 * q4 + i;
-      const uint32_t code = lm_code<W>(__uint_as_float(y[kk]) * sv[i], ctx);
-      const int bit = stream_bit<ROLE, W>(32 * HALF + kk);
-      s[bit >> 5] |= code << (bit & 31);
-      if ((bit & 31) + W > 32) s[(bit >> 5) + 1] |= code >> (32 - (bit & 31));
+      const int jj = 32 * HALF + 4 * q4 + i;
+      uint32_t code = code_of(__uint_as_float(y[4 * q4 + i]) * sv[i], L);
+      if (ZMASK && sv[i] == 0.f) code = 0;  // zero vector (or zero group): codes 0
+      A[code_word<ROLE>(jj)] |= code << (8 * code_byte<ROLE>(jj));
     }
   }
 }
 
-// The lane's fields sit e*W (keys) or 2h*W (values) bits further up; the partner
-// lane holds the other fields of the same portions.  Each lane keeps half of the
-// stream (keys: portions g = 4e..4e+3, values: c = 2h, 2h+1) and stores it: 8W bytes.
-template <int ROLE, int W>
-__device__ __forceinline__ void code_store(uint32_t (&s)[32], uint32_t side, unsigned mask,
-                                           uint8_t* dst) {
-  const uint32_t sh = ROLE == 0 ? side * W : side * 2 * W;
+// Store 8 chunks of 8W bits (chunk k at bit 8W k): the lane's 8W bytes.
+template <int W>
+__device__ __forceinline__ void store_stream(const uint32_t (&clo)[8], const uint32_t (&chi)[8],
+                                             uint8_t* dst) {
+  uint32_t o[2 * W];
 #pragma unroll
-  for (int i = 4 * W - 1; i > 0; --i) s[i] = __funnelshift_l(s[i - 1], s[i], sh);
-  s[0] <<= sh;
-  uint32_t out[2 * W];
+  for (int i = 0; i < 2 * W; ++i) o[i] = 0;
 #pragma unroll
-  for (int i = 0; i < 2 * W; ++i) {
-    const uint32_t send = side ? s[i] : s[2 * W + i];
-    const uint32_t recv = __shfl_xor_sync(mask, send, ROLE == 0 ? 1 : 8);
-    out[i] = (side ? s[2 * W + i] : s[i]) | recv;
+  for (int k = 0; k < 8; ++k) {
+    const int bit = 8 * W * k, w0 = bit >> 5, sh = bit & 31;
+    if (sh == 0) {
+      o[w0] |= clo[k];
+      if (w0 + 1 < 2 * W) o[w0 + 1] |= chi[k];
+    } else {
+      o[w0] |= clo[k] << sh;
+      if (w0 + 1 < 2 * W) o[w0 + 1] |= (clo[k] >> (32 - sh)) | (chi[k] << sh);
+      if (w0 + 2 < 2 * W) o[w0 + 2] |= chi[k] >> (32 - sh);
+    }
   }
 #pragma unroll
   for (int i = 0; i < W; ++i)
-    *reinterpret_cast<uint2*>(dst + 8 * i) = make_uint2(out[2 * i], out[2 * i + 1]);
+    *reinterpret_cast<uint2*>(dst + 8 * i) = make_uint2(o[2 * i], o[2 * i + 1]);
 }
 
-template <int ROLE, int HALF>
-__device__ __forceinline__ void code_half_w(int w, const uint32_t (&y)[32], const float* sc,
-                                            const float* thr4, const CodeLutMeta* lm,
-                                            const float2* cells, uint32_t (&s)[32]) {
-#define GTQ_CASE(W)                                                              \
-  case W:                                                                        \
-    code_half<ROLE, W, HALF>(y, sc, code_ctx<W>(thr4, lm, cells), s);            \
-    break;
-  switch (w) {
-    GTQ_CASE(1) GTQ_CASE(2) GTQ_CASE(3) GTQ_CASE(4)
-    GTQ_CASE(5) GTQ_CASE(6) GTQ_CASE(7) GTQ_CASE(8)
+// Merge with the partner lane, compress the 64 kept codes to W bits each and store.
+__device__ __forceinline__ void pack_store(const uint32_t (&A)[16], const CodeLane& L,
+                                           uint32_t side, int partner_xor, uint8_t* dst,
+                                           bool store) {
+  uint32_t keep[8], recv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t send = side ? A[i] : A[8 + i];
+    keep[i] = side ? A[8 + i] : A[i];
+    recv[i] = __shfl_xor_sync(0xffffffffu, send, partner_xor);
+  }
+  uint32_t clo[8], chi[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t v[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * k + h;  // 4 consecutive codes of the stream, in stream order
+      const uint32_t x = __byte_perm(keep[i >> 1], recv[i >> 1], (i & 1) ? L.sel_odd : L.sel_even);
+      const uint32_t d0 = __dp4a(x, L.mA, 0u), d1 = __dp4a(x, L.mB, 0u);
+      v[h] = L.w == 8 ? x : d0 + d1 * L.m2;
+    }
+    clo[k] = v[0] | __funnelshift_lc(0u, v[1], L.s4);
+    chi[k] = __funnelshift_lc(v[1], 0u, L.s4);
+  }
+  if (!store) return;
+  switch (L.w) {
+    case 1: store_stream<1>(clo, chi, dst); break;
+    case 2: store_stream<2>(clo, chi, dst); break;
+    case 3: store_stream<3>(clo, chi, dst); break;
+    case 4: store_stream<4>(clo, chi, dst); break;
+    case 5: store_stream<5>(clo, chi, dst); break;
+    case 6: store_stream<6>(clo, chi, dst); break;
+    case 7: store_stream<7>(clo, chi, dst); break;
+    case 8: store_stream<8>(clo, chi, dst); break;
     default: break;
   }
-#undef GTQ_CASE
-}
-
-template <int ROLE>
-__device__ __forceinline__ void code_store_w(int w, uint32_t (&s)[32], uint32_t side,
-                                             unsigned mask, uint8_t* dst) {
-#define GTQ_CASE(W) case W: code_store<ROLE, W>(s, side, mask, dst); break;
-  switch (w) {
-    GTQ_CASE(1) GTQ_CASE(2) GTQ_CASE(3) GTQ_CASE(4)
-    GTQ_CASE(5) GTQ_CASE(6) GTQ_CASE(7) GTQ_CASE(8)
-    default: break;
-  }
-#undef GTQ_CASE
 }
 
 template <int ROLE>
@@ -338,9 +324,8 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
   const int head = blockIdx.y, bidx = head / a.hkv, hidx = head % a.hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* scale = reinterpret_cast<float*>(sm + kOffScale);
-  float* thr4 = reinterpret_cast<float*>(sm + kOffThr);
+  uint8_t* zflags = sm + kOffFlags;
   const CodeLutMeta* lut_meta = reinterpret_cast<const CodeLutMeta*>(sm + kOffLut);
-  const float2* lut_cells = reinterpret_cast<const float2*>(sm + kOffLut + 128);
   HeadMeta& m = *reinterpret_cast<HeadMeta*>(sm + kOffMeta);
   GatherInfo& gi = *reinterpret_cast<GatherInfo*>(sm + kOffInfo);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + kNumBars * 8);
@@ -364,7 +349,6 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     mbar_init(bar(kRBar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < 4) thr4[tid] = a.thr[tid];  // width 1 (one threshold), width 2 (three)
   for (int i = tid; i < (int)(kCodeLutBytes / 16); i += kTcThreads)
     reinterpret_cast<uint4*>(sm + kOffLut)[i] = reinterpret_cast<const uint4*>(a.code_lut)[i];
   if (ROLE == 0) {
@@ -502,60 +486,77 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
           a.packed + ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + (j >> 6))) * a.tile_bytes;
       const uint8_t* xt = sm + kOffA + st * kStageBytes;
       float* sc_par = scale + par * kMaxGroups * kScaleStride;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      // one group is complete: stored norm and scale of token j
-      auto finish = [&](int g) {
-        const float S = (a0 + a1) + (a2 + a3);
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      unsigned zero_any = 0;
+      // one group is complete: stored norm and scale of token j.  acc[i] holds
+      // `terms` exact squares summed in fp32; the root is correctly rounded.
+      auto finish = [&](int g, int terms) {
+        const float S = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        const float n = sqrtf(S);
         float r;
         asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(S));
-        const float n = S * r;
-        // relative error of n: at most (chunks + 1) roundings of the sum's 2^-24
-        // (halved by the root), the approximate reciprocal root and one product
-        const float delta = (float)(gi.grp_chunks[g] + 12) * 5.9604645e-8f;
+        // |n / ||x|| - 1| <= (terms + 2) / 2 + 1/2 units of 2^-24 (sum depth terms - 1 + 3,
+        // halved by the root, plus its rounding); lo / hi add one rounding each
+        const float delta = (0.5f * (float)terms + 4.f) * 5.9604645e-8f;
         const float lo = n * (1.f - delta), hi = n * (1.f + delta);
-        __half h = __ushort_as_half(0);
-        float sv = __int_as_float(0x7fc00000);  // NaN: zero vector, codes 0
-        bool amb = false;
+        const float sv_n = gi.sqrt_m[g] * r;  // scale of the codes (fp32, about 2^-22 relative)
+        uint16_t hb = 0, hl = 0, hh = 0;
+        float sv = 0.f;
+        int amb = 0;  // 1: fp16 rounding undecided, 2: overflow undecided
         if (S == 0.f) {
         } else if (lo > 65504.f) {
-          h = __ushort_as_half(0x7BFF);
+          hb = 0x7BFF;
           ovf = 1;
-          sv = gi.sqrt_m[g] * r;
-        } else if (hi <= 65504.f &&
-                   __half_as_ushort(__float2half_rn(lo)) == __half_as_ushort(__float2half_rn(hi))) {
-          h = __float2half_rn(n);
-          sv = gi.sqrt_m[g] * r;
+          sv = sv_n;
+        } else if (hi > 65504.f) {
+          amb = 2;
+          sv = sv_n;
         } else {
-          amb = true;
+          hl = __half_as_ushort(__float2half_rn(lo));
+          hh = __half_as_ushort(__float2half_rn(hi));
+          hb = hl;
+          sv = sv_n;
+          if (hl != hh) amb = 1;
         }
-        unsigned am = __ballot_sync(0xffffffffu, amb);
-        while (am) {  // fp64 sum of the exact squares for one token, the whole warp helping
+        zero_any |= __ballot_sync(0xffffffffu, S == 0.f);
+        unsigned am = __ballot_sync(0xffffffffu, amb != 0);
+        while (am) {  // exact decision from the fp64 sum of squares, the whole warp helping
           const int src = __ffs(am) - 1;
           am &= am - 1;
           const int jt = 32 * q + src;
-          double acc = 0.0;
+          double sq = 0.0;
           for (int rr = lane; rr < gi.grp_rows[g]; rr += 32) {
             const int d = gi.row_dim[gi.grp_row0[g] + rr];
             const __half x = *reinterpret_cast<const __half*>(
                 xt + (d >> 6) * 16384 + jt * 128 + ((((d >> 3) & 7) ^ (jt & 7)) << 4) + (d & 7) * 2);
             const double xd = (double)__half2float(x);
-            acc = fma(xd, xd, acc);
+            sq = fma(xd, xd, sq);
           }
 #pragma unroll
-          for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
           if (lane == src) {
-            const double n64 = sqrt(acc);
-            if (n64 > 65504.0) ovf = 1;
-            h = __double2half(n64 > 65504.0 ? 65504.0 : n64);
-            sv = (float)((double)gi.sqrt_m[g] / n64);
+            if (amb == 1 && hh == hl + 1) {
+              // n is between the two fp16 values: compare with their midpoint squared
+              // (12 significant bits, exact in fp64); a tie rounds to even
+              const double mid = 0.5 * ((double)__half2float(__ushort_as_half(hl)) +
+                                        (double)__half2float(__ushort_as_half(hh)));
+              const double m2 = mid * mid;
+              hb = sq > m2 ? hh : (sq < m2 ? hl : ((hl & 1) ? hh : hl));
+            } else {
+              const double n64 = sqrt(sq);
+              if (n64 > 65504.0) ovf = 1;
+              hb = __half_as_ushort(__double2half(n64 > 65504.0 ? 65504.0 : n64));
+            }
           }
         }
-        *reinterpret_cast<__half*>(tile_base + norm_off + g * 128 + npos) = h;
+        *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb;
         sc_par[g * kScaleStride + j] = sv;
       };
       if (ROLE == 0) {
         // group sums of squares from the gathered exact inputs, 8 columns per chunk
-        int cur = 0;
+        int cur = 0, terms = 0;
         for (int b = 0; b < n_chunks; b += 4) {
           uint32_t r[32];
           tc_ld32(trow + 8 * b, r);
@@ -565,20 +566,22 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
             if (b + k < n_chunks) {
               const int g = gi.chunk_group[b + k];
               if (g != cur) {
-                finish(cur);
-                a0 = a1 = a2 = a3 = 0.f;
+                finish(cur, terms);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
                 cur = g;
+                terms = 0;
               }
 #pragma unroll
-              for (int e = 0; e < 8; e += 4) {
-                const float x0 = __uint_as_float(r[8 * k + e]), x1 = __uint_as_float(r[8 * k + e + 1]);
-                const float x2 = __uint_as_float(r[8 * k + e + 2]), x3 = __uint_as_float(r[8 * k + e + 3]);
-                a0 = fmaf(x0, x0, a0); a1 = fmaf(x1, x1, a1); a2 = fmaf(x2, x2, a2); a3 = fmaf(x3, x3, a3);
+              for (int e = 0; e < 8; ++e) {
+                const float x = __uint_as_float(r[8 * k + e]);
+                acc[e] = fmaf(x, x, acc[e]);
               }
+              ++terms;
             }
           }
         }
-        if (gi.n_groups > 0) finish(cur);
+        if (gi.n_groups > 0) finish(cur, terms);
       } else {
         // values: one group of all 128 dims, straight from the fp16 tile (row j, 16-byte
         // chunk c at position c ^ (j % 8) of its 128-byte row)
@@ -590,13 +593,14 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
           const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
           const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&v.z));
           const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&v.w));
-          a0 = fmaf(f0.x, f0.x, a0); a1 = fmaf(f0.y, f0.y, a1);
-          a2 = fmaf(f1.x, f1.x, a2); a3 = fmaf(f1.y, f1.y, a3);
-          a0 = fmaf(f2.x, f2.x, a0); a1 = fmaf(f2.y, f2.y, a1);
-          a2 = fmaf(f3.x, f3.x, a2); a3 = fmaf(f3.y, f3.y, a3);
+          acc[0] = fmaf(f0.x, f0.x, acc[0]); acc[1] = fmaf(f0.y, f0.y, acc[1]);
+          acc[2] = fmaf(f1.x, f1.x, acc[2]); acc[3] = fmaf(f1.y, f1.y, acc[3]);
+          acc[4] = fmaf(f2.x, f2.x, acc[4]); acc[5] = fmaf(f2.y, f2.y, acc[5]);
+          acc[6] = fmaf(f3.x, f3.x, acc[6]); acc[7] = fmaf(f3.y, f3.y, acc[7]);
         }
-        finish(0);
+        finish(0, 16);
       }
+      if (lane == 0) zflags[par * 4 + q] = zero_any ? 1 : 0;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -610,9 +614,8 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     // ----------------------------------------------------------- code warps
     const int q = warp & 3, hc = (warp - 6) >> 2;
     const int c = 32 * q + lane;  // rotated coordinate = tensor-memory lane
-    int w, grp;
+    int w, grp, dst_off;
     uint32_t side;
-    int dst_off;
     if (ROLE == 0) {
       const int slot = c >> 1;
       w = slot < m.n_slots ? m.slot_width[slot] : 0;
@@ -625,7 +628,29 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       side = (uint32_t)((c >> 3) & 1);
       dst_off = 1024 * a.kb + 16 * a.vb * (8 * (c >> 4) + (c & 7)) + 8 * a.vb * (int)side;
     }
-    const unsigned mask = __match_any_sync(0xffffffffu, w);
+    CodeLane L;
+    {
+      const int wl = w > 0 ? w : 1;  // width-0 lanes run width 1 and store nothing
+      L.w = w;
+      L.inv = lut_meta->inv[wl];
+      L.cadd = lut_meta->cadd[wl];
+      L.lut_base = sb + kOffLut + kCodeLutHeader + 8u * (uint32_t)lut_meta->off[wl] - 8u * 0x4B000000u;
+      L.lo = 0x4B000000;
+      L.hi = 0x4B000000 + lut_meta->nmax[wl];
+      if (ROLE == 0) {  // stream quad = [E(u), O(u), E(u+1), O(u+1)], E = even coordinate
+        L.sel_even = side ? 0x1504u : 0x5140u;
+        L.sel_odd = side ? 0x3726u : 0x7362u;
+      } else {          // stream quad = [E(l0), E(l1), O(l0), O(l1)], E = dim with h = 0
+        L.sel_even = side ? 0x1054u : 0x5410u;
+        L.sel_odd = side ? 0x3276u : 0x7632u;
+      }
+      const uint32_t p = 1u << wl;
+      L.mA = 1u | ((p & 0xFFu) << 8);
+      L.mB = (1u << 16) | ((p & 0xFFu) << 24);
+      L.m2 = 1u << (2 * wl);
+      L.s4 = 4u * (uint32_t)wl;
+    }
+    const int partner_xor = ROLE == 0 ? 1 : 8;
     const uint32_t tcol = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * hc);
     int it = 0;
     for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
@@ -634,14 +659,18 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       if (!mbar_wait(bar(kCFull + ac), (it >> 1) & 1)) { failed = 1; break; }
       tc_fence_after();
       const float* sc = scale + (par * kMaxGroups + grp) * kScaleStride + 64 * hc;
-      uint32_t s[32];
+      const bool zmask = *reinterpret_cast<const uint32_t*>(zflags + par * 4) != 0;
+      uint32_t A[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] = 0;
+      for (int i = 0; i < 16; ++i) A[i] = 0;
       {
         uint32_t y[32];
         tc_ld32(tcol + (uint32_t)(ac * kD), y);
         tc_wait_ld();
-        code_half_w<ROLE, 0>(w, y, sc, thr4, lut_meta, lut_cells, s);
+        if (zmask)
+          code_half<ROLE, 0, true>(y, sc, L, A);
+        else
+          code_half<ROLE, 0, false>(y, sc, L, A);
       }
       {
         uint32_t y[32];
@@ -650,14 +679,17 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kCEmpty + ac));  // accumulator may be overwritten
-        code_half_w<ROLE, 1>(w, y, sc + 32, thr4, lut_meta, lut_cells, s);
+        if (zmask)
+          code_half<ROLE, 1, true>(y, sc + 32, L, A);
+        else
+          code_half<ROLE, 1, false>(y, sc + 32, L, A);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kSEmpty + par));  // scales read
+      if (lane == 0) mbar_arrive(bar(kSEmpty + par));  // scales and flags read
       uint8_t* dst = a.packed +
                      ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + hc)) * a.tile_bytes +
                      dst_off;
-      code_store_w<ROLE>(w, s, side, mask, dst);
+      pack_store(A, L, side, partner_xor, dst, w > 0);
     }
   }
   if (failed) atomicOr(a.status, kStatusTimeout);
@@ -692,54 +724,58 @@ __global__ void b_image_kernel(const float* __restrict__ rows, size_t row_stride
   }
 }
 
-// Cell of |z| in the code table: floor(|z| * inv) as an fp32 fma rounded toward
-// zero onto 2^23 (the same expression the quantizer evaluates).
-__device__ __forceinline__ uint32_t code_cell(float a, float inv) {
-  return __float_as_uint(__fmaf_rz(a, inv, 8388608.f)) - 0x4B000000u;
+// Raw cell bits of z in the code table: bits(fma(z, inv, cadd) rounded toward zero)
+// minus bits(2^23) (the same expression the quantizer evaluates).
+__device__ __forceinline__ int code_cell(float z, float inv, float cadd) {
+  return __float_as_int(__fmaf_rz(z, inv, cadd)) - 0x4B000000;
 }
 
-// Builds the code table of widths 3..8 from the fp32 thresholds (one thread).
+// Builds the code table of widths 1..8 from the fp32 thresholds (one thread).
 __global__ void code_lut_kernel(const float* __restrict__ thr, uint8_t* __restrict__ blob) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   CodeLutMeta* lm = reinterpret_cast<CodeLutMeta*>(blob);
-  float2* cells = reinterpret_cast<float2*>(blob + 128);
+  float2* cells = reinterpret_cast<float2*>(blob + kCodeLutHeader);
   for (int w = 0; w <= GTQ_MAX_BITS; ++w) {
     lm->inv[w] = 0.f;
+    lm->cadd[w] = 8388608.f;
     lm->off[w] = 0;
     lm->nmax[w] = 0;
   }
   int off = 0, ok = 1;
-  for (int w = 3; w <= GTQ_MAX_BITS && ok; ++w) {
+  for (int w = 1; w <= GTQ_MAX_BITS && ok; ++w) {
     const float* t = thr + thr_base(w);
-    const int H = 1 << (w - 1);  // t[H - 1] = 0; positive thresholds t[H .. 2H - 2]
-    float gap = INFINITY;
-    for (int k = H; k <= 2 * H - 2; ++k) gap = fminf(gap, t[k] - t[k - 1]);
+    const int nt = (1 << w) - 1;
+    float gap = 1.f;
+    for (int k = 1; k < nt; ++k) gap = fminf(gap, t[k] - t[k - 1]);
     const float inv = 1.f / (0.98f * gap);
-    const int n = (int)code_cell(t[2 * H - 2], inv) + 2;  // the last cell holds no threshold
-    if (off + n > kCodeLutEntries) {
+    const int kofs = 2 - (int)floorf(t[0] * inv);  // the lowest threshold lands in cell >= 1
+    const float cadd = 8388608.f + (float)kofs;
+    const int n = code_cell(t[nt - 1], inv, cadd) + 2;  // the last cell holds no threshold
+    if (code_cell(t[0], inv, cadd) < 1 || off + n > kCodeLutEntries) {
       ok = 0;
       break;
     }
     for (int i = 0; i < n; ++i) cells[off + i] = make_float2(INFINITY, __int_as_float(0));
-    for (int k = H; k <= 2 * H - 2; ++k) {
-      const uint32_t c = code_cell(t[k], inv);
+    for (int k = 0; k < nt; ++k) {
+      const int c = code_cell(t[k], inv, cadd);
       if (cells[off + c].x != INFINITY) ok = 0;
       cells[off + c].x = t[k];
     }
-    int below = 0, k = H;
+    int below = 0, k = 0;
     for (int i = 0; i < n; ++i) {
-      while (k <= 2 * H - 2 && (int)code_cell(t[k], inv) < i) {
+      while (k < nt && code_cell(t[k], inv, cadd) < i) {
         ++below;
         ++k;
       }
       cells[off + i].y = __int_as_float(below);
     }
     lm->inv[w] = inv;
+    lm->cadd[w] = cadd;
     lm->off[w] = off;
     lm->nmax[w] = n - 1;
     off += n;
   }
-  lm->ok = ok;
+  *reinterpret_cast<int*>(blob + kCodeLutOkOffset) = ok;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

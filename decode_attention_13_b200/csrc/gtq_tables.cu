@@ -284,9 +284,9 @@ int tables_for(int device, uint64_t seed, Tables* out) {
   if (e == cudaSuccess) e = build_code_lut(t.thr, t.code_lut, 0);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e == cudaSuccess) {
-    CodeLutMeta lm;
-    e = cudaMemcpy(&lm, t.code_lut, sizeof(lm), cudaMemcpyDeviceToHost);
-    if (e == cudaSuccess && lm.ok != 1) {
+    int ok = 0;
+    e = cudaMemcpy(&ok, t.code_lut + kCodeLutOkOffset, sizeof(ok), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && ok != 1) {
       cudaSetDevice(prev);
       set_last_error("code lookup table: two thresholds share a cell");
       return GTQ_ERR_CUDA;
