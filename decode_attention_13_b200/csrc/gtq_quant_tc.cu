@@ -7,7 +7,8 @@
 // thresholds below (sqrt(m)/n) (M_h k)_j, fp16(n) stored; values likewise with
 // one group of 128 and R_V.
 //
-// One launch; a CTA works on one head in one role (blockIdx.z: 0 keys, 1 values)
+// One launch; a CTA works on one head in one role (keys or values; a head's CTAs
+// are shared between the roles by their cost per tile)
 // and walks 128-token tiles that lie inside the tokens being written.  Per tile:
 //   * code GEMM   D_c[coord][token] = R . X^T with R = M_h (keys) or R_V (values)
 //                 split into fp16 hi + lo parts (A operand, resident in shared
@@ -25,10 +26,10 @@
 //
 // Norms: the fp32 sum of exact squares has a rigorous relative error bound;
 // when fp16 rounding of every value inside the bound agrees, that is the stored
-// norm, otherwise (about 0.1-0.4 % of norms) the warp recomputes the sum in fp64
-// from the fp16 tile in shared memory.  Scales for the codes come from the same
-// norm (fp32 division).  Zero vectors get a NaN scale so that every code
-// comparison is false and the codes are 0.
+// norm, otherwise (about 0.1-0.4 % of norms) the warp decides it exactly from the
+// fp64 sum of squares of the fp16 tile in shared memory.  Scales for the codes
+// come from the same sum (approximate reciprocal root).  A tile that holds a zero
+// vector or group is flagged, and its codes are masked to 0.
 // Waits are bounded; on expiry the status word gets GTQ_ERR_TIMEOUT's bit.
 #include <cuda.h>
 
@@ -44,6 +45,7 @@ constexpr int kTcWarps = 14;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kMTile = 128;          // tokens per MMA tile (= 2 packed tiles)
 constexpr int kStages = 3;           // input tile stages
+constexpr int kKeyShare = 67;        // percent of a head's CTAs that quantize keys
 constexpr uint64_t kTcWaitNs = 2000000000ull;  // bound of every barrier wait
 
 constexpr int kMaxPRows = 176;       // 128 dims + at most 6 padding rows for each of 8 groups
@@ -108,6 +110,7 @@ struct TcArgs {
   int tile_bytes;
   int kb, vb, pairing, hkv;
   int64_t mt0, mt1;       // MMA tiles [mt0, mt1) of every head
+  int ctas_k, ctas_v;     // CTAs per head of each role (blockIdx.x < ctas_k: keys)
   int* status;
 };
 
@@ -317,7 +320,8 @@ __device__ __forceinline__ void pack_store(const uint32_t (&A)[16], const CodeLa
 }
 
 template <int ROLE>
-__device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a) {
+__device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a, int cta,
+                                        int n_cta) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = su32(sm);
@@ -420,7 +424,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       mbar_expect_tx(bar(kRBar), kBBytes);
       bulk_load(sb + kOffB, rsrc, kBBytes, bar(kRBar));
       int it = 0;
-      for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
+      for (int64_t t = cta; t < n_mt; t += n_cta, ++it) {
         const int st = it % kStages;
         if (!mbar_wait(bar(kEmpty + st), ((it / kStages) & 1) ^ 1)) { failed = 1; break; }
         const uint32_t dst = sb + kOffA + st * kStageBytes;
@@ -437,7 +441,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       const uint32_t idc = idesc_f16(kD), idp = idesc_f16(n_rows);
       const uint32_t p_atom = (uint32_t)n_rows * 128;
       int it = 0;
-      for (int64_t t = blockIdx.x; t < n_mt && !failed; t += gridDim.x, ++it) {
+      for (int64_t t = cta; t < n_mt && !failed; t += n_cta, ++it) {
         const int st = it % kStages, ac = it & 1;
         if (!mbar_wait(bar(kFull + st), (it / kStages) & 1)) { failed = 1; break; }
         const uint32_t x_base = sb + kOffA + st * kStageBytes;
@@ -472,8 +476,16 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     const int norm_off = ROLE == 0 ? 1024 * (a.kb + a.vb) + 128 : 1024 * (a.kb + a.vb);
     const int jj = j & 63, npos = 2 * ((jj & 7) * 8 + (jj >> 3));
     const int n_chunks = gi.n_chunks;
+    uint32_t cgw[(kMaxChunks + 7) / 8];  // group of chunk c: 4 bits at (c % 8) * 4 of word c / 8
+#pragma unroll
+    for (int w = 0; w < (kMaxChunks + 7) / 8; ++w) {
+      cgw[w] = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (8 * w + k < n_chunks) cgw[w] |= (uint32_t)gi.chunk_group[8 * w + k] << (4 * k);
+    }
     int ovf = 0, it = 0;
-    for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
+    for (int64_t t = cta; t < n_mt; t += n_cta, ++it) {
       const int st = it % kStages, par = it & 1;
       if (ROLE == 0) {
         if (!mbar_wait(bar(kPFull), it & 1)) { failed = 1; break; }
@@ -486,105 +498,56 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
           a.packed + ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + (j >> 6))) * a.tile_bytes;
       const uint8_t* xt = sm + kOffA + st * kStageBytes;
       float* sc_par = scale + par * kMaxGroups * kScaleStride;
+      // group sums of exact squares in fp32 (eight accumulators; a group's index is
+      // uniform, so its sum lands in a register through predicated moves)
+      float Sg[kMaxGroups];
+#pragma unroll
+      for (int g = 0; g < kMaxGroups; ++g) Sg[g] = 0.f;
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      unsigned zero_any = 0;
-      // one group is complete: stored norm and scale of token j.  acc[i] holds
-      // `terms` exact squares summed in fp32; the root is correctly rounded.
-      auto finish = [&](int g, int terms) {
+      auto put = [&](int g) {
         const float S = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        const float n = sqrtf(S);
-        float r;
-        asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(S));
-        // |n / ||x|| - 1| <= (terms + 2) / 2 + 1/2 units of 2^-24 (sum depth terms - 1 + 3,
-        // halved by the root, plus its rounding); lo / hi add one rounding each
-        const float delta = (0.5f * (float)terms + 4.f) * 5.9604645e-8f;
-        const float lo = n * (1.f - delta), hi = n * (1.f + delta);
-        const float sv_n = gi.sqrt_m[g] * r;  // scale of the codes (fp32, about 2^-22 relative)
-        uint16_t hb = 0, hl = 0, hh = 0;
-        float sv = 0.f;
-        int amb = 0;  // 1: fp16 rounding undecided, 2: overflow undecided
-        if (S == 0.f) {
-        } else if (lo > 65504.f) {
-          hb = 0x7BFF;
-          ovf = 1;
-          sv = sv_n;
-        } else if (hi > 65504.f) {
-          amb = 2;
-          sv = sv_n;
-        } else {
-          hl = __half_as_ushort(__float2half_rn(lo));
-          hh = __half_as_ushort(__float2half_rn(hi));
-          hb = hl;
-          sv = sv_n;
-          if (hl != hh) amb = 1;
-        }
-        zero_any |= __ballot_sync(0xffffffffu, S == 0.f);
-        unsigned am = __ballot_sync(0xffffffffu, amb != 0);
-        while (am) {  // exact decision from the fp64 sum of squares, the whole warp helping
-          const int src = __ffs(am) - 1;
-          am &= am - 1;
-          const int jt = 32 * q + src;
-          double sq = 0.0;
-          for (int rr = lane; rr < gi.grp_rows[g]; rr += 32) {
-            const int d = gi.row_dim[gi.grp_row0[g] + rr];
-            const __half x = *reinterpret_cast<const __half*>(
-                xt + (d >> 6) * 16384 + jt * 128 + ((((d >> 3) & 7) ^ (jt & 7)) << 4) + (d & 7) * 2);
-            const double xd = (double)__half2float(x);
-            sq = fma(xd, xd, sq);
-          }
 #pragma unroll
-          for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-          if (lane == src) {
-            if (amb == 1 && hh == hl + 1) {
-              // n is between the two fp16 values: compare with their midpoint squared
-              // (12 significant bits, exact in fp64); a tie rounds to even
-              const double mid = 0.5 * ((double)__half2float(__ushort_as_half(hl)) +
-                                        (double)__half2float(__ushort_as_half(hh)));
-              const double m2 = mid * mid;
-              hb = sq > m2 ? hh : (sq < m2 ? hl : ((hl & 1) ? hh : hl));
-            } else {
-              const double n64 = sqrt(sq);
-              if (n64 > 65504.0) ovf = 1;
-              hb = __half_as_ushort(__double2half(n64 > 65504.0 ? 65504.0 : n64));
-            }
-          }
-        }
-        *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb;
-        sc_par[g * kScaleStride + j] = sv;
+        for (int gg = 0; gg < kMaxGroups; ++gg)
+          if (gg == g) Sg[gg] = S;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       };
+      int ng;
       if (ROLE == 0) {
-        // group sums of squares from the gathered exact inputs, 8 columns per chunk
-        int cur = 0, terms = 0;
-        for (int b = 0; b < n_chunks; b += 4) {
-          uint32_t r[32];
-          tc_ld32(trow + 8 * b, r);
+        // gathered exact inputs, 8 columns per chunk, 8 chunks per wait
+        ng = gi.n_groups;
+        int cur = 0;
+#pragma unroll
+        for (int w = 0; w < (kMaxChunks + 7) / 8; ++w) {
+          const int b = 8 * w;
+          if (b >= n_chunks) break;
+          uint32_t r0[32], r1[32];
+          tc_ld32(trow + 8 * b, r0);
+          tc_ld32(trow + 8 * b + 32, r1);
           tc_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 8; ++k) {
             if (b + k < n_chunks) {
-              const int g = gi.chunk_group[b + k];
+              const int g = (int)((cgw[w] >> (4 * k)) & 15u);
               if (g != cur) {
-                finish(cur, terms);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                put(cur);
                 cur = g;
-                terms = 0;
               }
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const float x = __uint_as_float(r[8 * k + e]);
+                const float x = __uint_as_float(k < 4 ? r0[8 * k + e] : r1[8 * (k - 4) + e]);
                 acc[e] = fmaf(x, x, acc[e]);
               }
-              ++terms;
             }
           }
         }
-        if (gi.n_groups > 0) finish(cur, terms);
+        if (ng > 0) put(cur);
       } else {
         // values: one group of all 128 dims, straight from the fp16 tile (row j, 16-byte
         // chunk c at position c ^ (j % 8) of its 128-byte row)
+        ng = 1;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const uint4 v = *reinterpret_cast<const uint4*>(
@@ -598,8 +561,81 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
           acc[4] = fmaf(f2.x, f2.x, acc[4]); acc[5] = fmaf(f2.y, f2.y, acc[5]);
           acc[6] = fmaf(f3.x, f3.x, acc[6]); acc[7] = fmaf(f3.y, f3.y, acc[7]);
         }
-        finish(0, 16);
+        put(0);
       }
+      // every group's norm at once (independent chains).  acc[i] held `terms` exact
+      // squares: |n / ||x|| - 1| <= (terms + 2) / 2 + 1/2 units of 2^-24 (sum depth
+      // terms - 1 + 3, halved by the root, plus its rounding); lo / hi add one each
+      uint16_t hb[kMaxGroups], hl[kMaxGroups], hh[kMaxGroups];
+      float sv[kMaxGroups];
+      unsigned ambm = 0, zm = 0;  // 2 bits per group: 1 fp16 rounding undecided, 2 overflow undecided
+#pragma unroll
+      for (int g = 0; g < kMaxGroups; ++g) {  // all eight computed (unused groups have S = 0)
+        const float S = Sg[g];
+        const int terms = ROLE == 0 ? gi.grp_chunks[g] : 16;
+        const float n = sqrtf(S);
+        float r;
+        asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(S));
+        const float delta = (0.5f * (float)terms + 4.f) * 5.9604645e-8f;
+        const float lo = n * (1.f - delta), hi = n * (1.f + delta);
+        const bool live = g < ng;
+        const bool zero = S == 0.f, over = lo > 65504.f, strad = !over && hi > 65504.f;
+        const uint16_t l16 = __half_as_ushort(__float2half_rn(fminf(lo, 65504.f)));
+        const uint16_t h16 = __half_as_ushort(__float2half_rn(fminf(hi, 65504.f)));
+        hl[g] = l16;
+        hh[g] = h16;
+        hb[g] = zero ? (uint16_t)0 : (over ? (uint16_t)0x7BFF : l16);
+        sv[g] = zero ? 0.f : gi.sqrt_m[g] * r;  // scale of the codes (fp32, about 2^-22 relative)
+        if (live) {
+          zm |= zero ? 1u : 0u;
+          ovf |= over ? 1 : 0;
+          ambm |= (zero || over) ? 0u : (strad ? 2u : (l16 != h16 ? 1u : 0u)) << (2 * g);
+        }
+      }
+      const unsigned zero_any = __ballot_sync(0xffffffffu, zm != 0);
+      if (__ballot_sync(0xffffffffu, ambm != 0)) {
+#pragma unroll
+        for (int g = 0; g < kMaxGroups; ++g) {
+          if (g >= ng) break;
+          const unsigned amb_g = (ambm >> (2 * g)) & 3u;
+          unsigned am = __ballot_sync(0xffffffffu, amb_g != 0);
+          while (am) {  // exact decision from the fp64 sum of squares, the whole warp helping
+            const int src = __ffs(am) - 1;
+            am &= am - 1;
+            const int jt = 32 * q + src;
+            double sq = 0.0;
+            for (int rr = lane; rr < gi.grp_rows[g]; rr += 32) {
+              const int d = gi.row_dim[gi.grp_row0[g] + rr];
+              const __half x = *reinterpret_cast<const __half*>(
+                  xt + (d >> 6) * 16384 + jt * 128 + ((((d >> 3) & 7) ^ (jt & 7)) << 4) + (d & 7) * 2);
+              const double xd = (double)__half2float(x);
+              sq = fma(xd, xd, sq);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (lane == src) {
+              if (amb_g == 1 && hh[g] == hl[g] + 1) {
+                // n is between the two fp16 values: compare with their midpoint squared
+                // (12 significant bits, exact in fp64); a tie rounds to even
+                const double mid = 0.5 * ((double)__half2float(__ushort_as_half(hl[g])) +
+                                          (double)__half2float(__ushort_as_half(hh[g])));
+                const double m2 = mid * mid;
+                hb[g] = sq > m2 ? hh[g] : (sq < m2 ? hl[g] : ((hl[g] & 1) ? hh[g] : hl[g]));
+              } else {
+                const double n64 = sqrt(sq);
+                if (n64 > 65504.0) ovf = 1;
+                hb[g] = __half_as_ushort(__double2half(n64 > 65504.0 ? 65504.0 : n64));
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < kMaxGroups; ++g)
+        if (g < ng) {
+          *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb[g];
+          sc_par[g * kScaleStride + j] = sv[g];
+        }
       if (lane == 0) zflags[par * 4 + q] = zero_any ? 1 : 0;
       tc_fence_before();
       __syncwarp();
@@ -653,7 +689,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     const int partner_xor = ROLE == 0 ? 1 : 8;
     const uint32_t tcol = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * hc);
     int it = 0;
-    for (int64_t t = blockIdx.x; t < n_mt; t += gridDim.x, ++it) {
+    for (int64_t t = cta; t < n_mt; t += n_cta, ++it) {
       const int ac = it & 1, par = it & 1;
       if (!mbar_wait(bar(kSFull + par), (it >> 1) & 1)) { failed = 1; break; }
       if (!mbar_wait(bar(kCFull + ac), (it >> 1) & 1)) { failed = 1; break; }
@@ -701,10 +737,10 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
 __global__ void __launch_bounds__(kTcThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv, TcArgs a) {
-  if (blockIdx.z == 0)
-    tc_role<0>(&tmk, a);
+  if ((int)blockIdx.x < a.ctas_k)
+    tc_role<0>(&tmk, a, blockIdx.x, a.ctas_k);
   else
-    tc_role<1>(&tmv, a);
+    tc_role<1>(&tmv, a, blockIdx.x - a.ctas_k, a.ctas_v);
 }
 
 // R image of a 128 x 128 matrix (rows = output coordinate, cols = input dim):
@@ -850,12 +886,16 @@ cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, 
   a.mt1 = mt1;
   a.status = p->d_status;
   const int64_t n_mt = mt1 - mt0;
-  const int per_head =
-      (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, p->n_sms / std::max(1, 2 * p->n_heads)));
+  // SMs per head are shared between the roles by their measured cost per tile
+  // (a key tile costs about twice a value tile); every CTA keeps one head
+  const int per_head = std::max(2, p->n_sms / std::max(1, p->n_heads));
+  a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, (per_head * kKeyShare + 99) / 100));
+  a.ctas_v = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, per_head - a.ctas_k));
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
   if (e != cudaSuccess) return e;
-  quantize_tc_kernel<<<dim3(per_head, p->n_heads, 2), kTcThreads, kTcSmem, s>>>(maps[0], maps[1], a);
+  quantize_tc_kernel<<<dim3(a.ctas_k + a.ctas_v, p->n_heads), kTcThreads, kTcSmem, s>>>(maps[0],
+                                                                                        maps[1], a);
   return cudaGetLastError();
 }
 
