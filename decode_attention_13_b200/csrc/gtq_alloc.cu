@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
                                                    const double* __restrict__ energy,
                                                    const double* __restrict__ rot_k, int pairing,
                                                    HeadMeta* __restrict__ meta_out,
-                                                   float* __restrict__ mrow) {
+                                                   float* __restrict__ mrow,
+                                                   float* __restrict__ mrow_t) {
   const int head = blockIdx.x;
   __shared__ HeadMeta m;
   __shared__ uint8_t grp_blocks[kMaxGroups][kBlocks];
@@ -214,6 +215,7 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
   // key rotation rows: M_h[pos][dim], pos = 2 * slot + e  <->  row r = 2 (slot - first) + e of R_m
   const int pos = threadIdx.x;
   float* row = mrow + ((size_t)head * kD + pos) * kD;
+  float* col = mrow_t + (size_t)head * kD * kD + pos;  // M_h^T[dim][pos]
   for (int dd = 0; dd < kD; ++dd) row[dd] = 0.f;
   const int slot = pos >> 1;
   if (slot < m.n_slots) {
@@ -229,6 +231,7 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
       row[dim] = (float)R[c];
     }
   }
+  for (int dd = 0; dd < kD; ++dd) col[(size_t)dd * kD] = row[dd];
   if (threadIdx.x == 0) meta_out[head] = m;
 }
 
@@ -262,7 +265,7 @@ cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s) {
       p->d_bits);
   if (p->cfg.head_dim == kD) {
     meta_kernel<<<p->n_heads, 128, 0, s>>>(p->d_bits, p->d_energy, p->tab.rot_k,
-                                           p->cfg.rope_pairing, p->d_meta, p->d_mrow);
+                                           p->cfg.rope_pairing, p->d_meta, p->d_mrow, p->d_mrow_t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return build_b_images(p->d_mrow, p->n_heads, (size_t)kD * kD, p->d_bimg, s);

@@ -50,6 +50,7 @@ void release(gtq_plan* p) {
   cudaFree(p->d_bits);
   cudaFree(p->d_meta);
   cudaFree(p->d_mrow);
+  cudaFree(p->d_mrow_t);
   cudaFree(p->d_bimg);
   cudaFree(p->d_qrot);
   cudaFree(p->d_partials);
@@ -89,6 +90,7 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   alloc((void**)&p->d_bits, H * p->n_blocks);
   alloc((void**)&p->d_meta, H * sizeof(HeadMeta));
   alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
+  alloc((void**)&p->d_mrow_t, H * kD * kD * sizeof(float));
   if (cfg->head_dim == kD) alloc((void**)&p->d_bimg, H * b_image_bytes());
   alloc((void**)&p->d_qrot, H * 8 * kD * sizeof(float));
   alloc((void**)&p->d_partials, H * kPartialSlots * 8 * kPartialStride * sizeof(float));

@@ -25,16 +25,16 @@
 namespace gtq {
 namespace {
 
-constexpr int kWarps = 12;  // one CTA per SM: up to 12 warps, 2 private tile stages each
-constexpr int kStages = 2;
+constexpr int kPairs = 8;  // one CTA per SM: up to 8 warp pairs, 2 tile stages per pair
+constexpr int kWarps = 2 * kPairs;
+constexpr int kMaxStages = 3;  // tile stages per warp pair (3 when 8 pairs fit, else 2)
 constexpr unsigned kSpinLimit = 1u << 26;
-constexpr unsigned kBarrierSpinLimit = 1u << 24;  // x >= 64 ns: over a second
 
 struct DecodeArgs {
   const uint8_t* packed;
   const HeadMeta* meta;
   const void* q;        // [B][Hq][128] fp16 or fp32 (q_fp32)
-  const float* mrow;    // [heads][128][128] key rotation rows in packed order
+  const float* mrow_t;  // [heads][128][128] key rotation, transposed: [dim][packed position]
   const float* rot_v;   // R_V [128][128]
   float* out;           // [B][Hq][128]
   const uint4* dec_image;  // lookup tables (kDecodeImageBytes)
@@ -48,6 +48,8 @@ struct DecodeArgs {
   int tile_bytes;
   int kb, vb;
   int splits;
+  int stages;         // tile stages per warp pair
+  int rot_off;        // byte offset of the setup scratch in the stage area
   int64_t tiles_T;    // ceil(T / 64)
 };
 
@@ -59,14 +61,32 @@ __device__ inline void mbar_init(uint64_t* bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 
-__device__ inline void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing bytes on the mbarrier
+__device__ inline void bulk_copy(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
           "r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// L2 policy for the packed cache: streamed once per call, evicted first, so
+// that it does not push the tables, rotations and code out of L2
+__device__ inline uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// one packed tile: arm the stage's mbarrier with the byte count, then copy
+__device__ inline void tile_load(void* dst, const void* src, unsigned bytes, uint64_t* bar,
+                                 uint64_t policy) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -110,29 +130,31 @@ __device__ inline uint32_t pack_half2(__half lo, __half hi) {
 }
 
 // ---------------------------------------------------------------------------
-// Code -> fp16 lookups.
-//
-// Pair tables (widths 1..3, fp16 hi parts): entry idx = c0 | c1 << w holds the
-// half2 (cb[c0], cb[c1]); every lane has its own copy (word idx * 32 + lane), so
-// a warp-wide lookup never has a bank conflict.  Width w's table sits at byte
-// offset kPairOff(w), chosen so that offset | idx * 128 | lane * 4 needs no add.
-// Single-code tables (widths 1..8, 2^w entries of 32 bits: fp16 hi part in the
-// low half, fp16 lo part in the high half): at byte offset 2048 - 2^(w+3) inside
-// a 2 KB region, so offset | code * 4 needs no add; widths up to 5 occupy at
-// most 32 banks and never conflict.
+// Code -> fp16 lookups (table layout: gtq_internal.h).  Every lookup address is
+// "region offset (an immediate) + (field << k | lane * 4)": one shift and one
+// mask-or per lookup.  Widths 1..3 use lane-private pair tables (one lookup per
+// half2), widths 4..6 lane-private single-code tables, widths 7..8 and the lo
+// parts of narrow split groups one shared single-code table.
 // ---------------------------------------------------------------------------
 
+static_assert(sizeof(HeadMeta) % 16 == 0, "metadata is bulk-copied");
+
 struct DecodeSmem {
-  uint32_t pair[kPairBytes / 4];  // pair and single tables: one contiguous image
-  uint32_t single[kSingleBytes / 4];
+  uint32_t tab[kDecodeImageBytes / 4];
   uint4 qf[kMaxKt][32];  // per k-tile & lane: hi(slot A), hi(slot B), lo(A), lo(B)
-  HeadMeta meta;
-  uint64_t bar[kWarps][kStages];
+  alignas(16) HeadMeta meta;
+  uint64_t setup_bar;              // lookup tables and metadata loaded
+  uint64_t bar[kPairs][kMaxStages];   // tile loaded (bulk copy complete)
+  unsigned done[kPairs][kMaxStages];  // releases of a stage by the two warps of its pair
   float wm[kWarps][8], wl[kWarps][8], wsc[kWarps][8], hm[8], hl[8];
-  float qs[8][kD];  // queries of this KV head, then the merged o_rot
-  float qr[8][kD];  // rotated, scaled queries
+  alignas(16) float qs[8][kD];  // queries of this KV head, then the merged o_rot
+  alignas(16) float qr[8][kD];  // rotated, scaled queries
   int flag;
 };
+// vector (16-byte) and bulk-copy accesses
+static_assert(offsetof(DecodeSmem, qf) % 16 == 0 && offsetof(DecodeSmem, meta) % 16 == 0 &&
+                  offsetof(DecodeSmem, qs) % 16 == 0 && offsetof(DecodeSmem, qr) % 16 == 0,
+              "shared-memory alignment");
 
 // bits [P, P + N) of the little-endian bit string x[], moved to bit S, masked, OR orv
 template <int P, int N, int S>
@@ -150,43 +172,50 @@ __device__ __forceinline__ uint32_t fld(const uint32_t* x, uint32_t orv) {
   return (v & mask) | orv;
 }
 
-__device__ __forceinline__ uint32_t lds32(const DecodeSmem& s, uint32_t byte_off) {
-  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(s.pair) + byte_off);
-}
-__device__ __forceinline__ uint32_t lds_single(const DecodeSmem& s, uint32_t byte_off) {
-  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(s.single) + byte_off);
+template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds_tab(const DecodeSmem& s, uint32_t idx) {
+  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(s.tab) + OFF + idx);
 }
 
-// half2 of codes (2x, 2x+1), width W, from the bit string x (pair at bits [2xW, 2xW + 2W))
+// hi|lo word (fp16 hi in the low half) of the code of width W at bits [P, P + W)
+template <int W, int P>
+__device__ __forceinline__ uint32_t single_code(const DecodeSmem& s, const uint32_t* x, uint32_t lane4) {
+  if constexpr (W >= 4 && W <= 6)
+    return lds_tab<kLaneSingleOff(W)>(s, fld<P, W, 7>(x, lane4));
+  else
+    return lds_tab<kSharedSingles + kSingleOff(W)>(s, fld<P, W, 2>(x, 0u));
+}
+
+// half2 (hi parts) of codes (2X, 2X + 1), width W, from the bit string x
 template <int W, int X>
-__device__ __forceinline__ uint32_t pair_hi(const DecodeSmem& s, const uint32_t* x, uint32_t lane_pair) {
+__device__ __forceinline__ uint32_t pair_hi(const DecodeSmem& s, const uint32_t* x, uint32_t lane4) {
   if constexpr (W <= 3) {
-    return lds32(s, fld<2 * X * W, 2 * W, 7>(x, lane_pair));
+    return lds_tab<kPairOff(W)>(s, fld<2 * X * W, 2 * W, 7>(x, lane4));
   } else {
-    const uint32_t e0 = lds_single(s, fld<2 * X * W, W, 2>(x, kSingleOff(W)));
-    const uint32_t e1 = lds_single(s, fld<(2 * X + 1) * W, W, 2>(x, kSingleOff(W)));
+    const uint32_t e0 = single_code<W, 2 * X * W>(s, x, lane4);
+    const uint32_t e1 = single_code<W, (2 * X + 1) * W>(s, x, lane4);
     return __byte_perm(e0, e1, 0x5410);
   }
 }
-// hi and lo half2 of codes (2x, 2x+1) from the combined single-code table
+// hi and lo half2 of codes (2X, 2X + 1) from the single-code tables
 template <int W, int X>
-__device__ __forceinline__ void pair_hilo(const DecodeSmem& s, const uint32_t* x, uint32_t& hi,
-                                          uint32_t& lo) {
-  const uint32_t e0 = lds_single(s, fld<2 * X * W, W, 2>(x, kSingleOff(W)));
-  const uint32_t e1 = lds_single(s, fld<(2 * X + 1) * W, W, 2>(x, kSingleOff(W)));
+__device__ __forceinline__ void pair_hilo(const DecodeSmem& s, const uint32_t* x, uint32_t lane4,
+                                          uint32_t& hi, uint32_t& lo) {
+  const uint32_t e0 = single_code<W, 2 * X * W>(s, x, lane4);
+  const uint32_t e1 = single_code<W, (2 * X + 1) * W>(s, x, lane4);
   hi = __byte_perm(e0, e1, 0x5410);
   lo = __byte_perm(e0, e1, 0x7632);
 }
 
-// The 16w-bit portion of one key slot for this lane (tokens g + 8u, u = 0..7),
-// realigned to bit 0 of x[] (portions start at an even byte).
-template <int W>
-struct KeyWords {
-  static constexpr int NW = (16 * W + 31) / 32 + 1;
+// NB bits of packed codes starting at byte byte_off of tile, realigned to bit 0
+// of x[] (x holds NB bits plus up to 24 bits of what follows).
+template <int NB>
+struct Bits {
+  static constexpr int NW = (NB + 31) / 32 + 1;
   uint32_t x[NW];
   __device__ __forceinline__ void load(const uint8_t* tile, int byte_off) {
     const uint32_t* wp = reinterpret_cast<const uint32_t*>(tile + (byte_off & ~3));
-    const uint32_t sh = (byte_off & 2) << 3;  // 0 or 16
+    const uint32_t sh = (uint32_t)(byte_off & 3) << 3;
 #pragma unroll
     for (int i = 0; i < NW; ++i) x[i] = wp[i];
 #pragma unroll
@@ -194,44 +223,46 @@ struct KeyWords {
   }
 };
 
-// One decode k-tile of a group of width W: 8 slots x 16 coords; this lane's
-// slots are first + t (A-fragment regs 0/1) and first + t + 4 (regs 2/3).
-// Slots past the group's run read unrelated bits; their q is zero.  When the
-// run has at most 4 slots the second half is all padding and is skipped.
-// SPLIT adds the hi.lo and lo.hi terms of the split fp16 product (same accumulator).
+// One decode k-tile of a group of width W for this warp's 32 tokens: 8 slots x
+// 16 coords; this lane's slots are first + t (A-fragment regs 0/1) and
+// first + t + 4 (regs 2/3), its tokens g + 8u for the warp's u = 4h .. 4h + 3,
+// i.e. 8W bits of each slot's 16W-bit lane portion.  Slots past the group's
+// run read unrelated bits; their q is zero.  When the run has at most 4 slots
+// the second half is all padding and is skipped.  SPLIT adds the hi.lo and
+// lo.hi terms of the split fp16 product (same accumulator).
 template <int W, bool SPLIT>
 __device__ __forceinline__ void ktile_step(const DecodeSmem& s, const uint8_t* tile, int koff_a,
-                                           bool has_b, uint32_t lane_pair, const uint4& bq,
-                                           float (&C)[4][4]) {
-  constexpr bool kCombined = W >= 4;  // single-code table: hi and lo from one load
-  KeyWords<W> ka, kb;
+                                           bool has_b, uint32_t lane4, const uint4& bq,
+                                           float (&C)[2][4]) {
+  constexpr bool kCombined = W >= 4;  // single-code tables: hi and lo from one load
+  Bits<8 * W> ka, kb;
   ka.load(tile, koff_a);
   if (has_b) kb.load(tile, koff_a + 64 * W);
 #define GTQ_MT(MT)                                                                   \
   {                                                                                  \
     uint32_t ah[4], al[4];                                                           \
     if constexpr (kCombined) {                                                       \
-      pair_hilo<W, 2 * (MT)>(s, ka.x, ah[0], al[0]);                                 \
-      pair_hilo<W, 2 * (MT) + 1>(s, ka.x, ah[1], al[1]);                             \
+      pair_hilo<W, 2 * (MT)>(s, ka.x, lane4, ah[0], al[0]);                          \
+      pair_hilo<W, 2 * (MT) + 1>(s, ka.x, lane4, ah[1], al[1]);                      \
       if (has_b) {                                                                   \
-        pair_hilo<W, 2 * (MT)>(s, kb.x, ah[2], al[2]);                               \
-        pair_hilo<W, 2 * (MT) + 1>(s, kb.x, ah[3], al[3]);                           \
+        pair_hilo<W, 2 * (MT)>(s, kb.x, lane4, ah[2], al[2]);                        \
+        pair_hilo<W, 2 * (MT) + 1>(s, kb.x, lane4, ah[3], al[3]);                    \
       } else {                                                                       \
         ah[2] = ah[3] = al[2] = al[3] = 0u;                                          \
       }                                                                              \
     } else {                                                                         \
-      ah[0] = pair_hi<W, 2 * (MT)>(s, ka.x, lane_pair);                              \
-      ah[1] = pair_hi<W, 2 * (MT) + 1>(s, ka.x, lane_pair);                          \
-      ah[2] = has_b ? pair_hi<W, 2 * (MT)>(s, kb.x, lane_pair) : 0u;                 \
-      ah[3] = has_b ? pair_hi<W, 2 * (MT) + 1>(s, kb.x, lane_pair) : 0u;             \
+      ah[0] = pair_hi<W, 2 * (MT)>(s, ka.x, lane4);                                  \
+      ah[1] = pair_hi<W, 2 * (MT) + 1>(s, ka.x, lane4);                              \
+      ah[2] = has_b ? pair_hi<W, 2 * (MT)>(s, kb.x, lane4) : 0u;                     \
+      ah[3] = has_b ? pair_hi<W, 2 * (MT) + 1>(s, kb.x, lane4) : 0u;                 \
       if constexpr (SPLIT) {                                                         \
         uint32_t dummy;                                                              \
-        pair_hilo<W, 2 * (MT)>(s, ka.x, dummy, al[0]);                               \
-        pair_hilo<W, 2 * (MT) + 1>(s, ka.x, dummy, al[1]);                           \
+        pair_hilo<W, 2 * (MT)>(s, ka.x, lane4, dummy, al[0]);                        \
+        pair_hilo<W, 2 * (MT) + 1>(s, ka.x, lane4, dummy, al[1]);                    \
         al[2] = al[3] = 0u;                                                          \
         if (has_b) {                                                                 \
-          pair_hilo<W, 2 * (MT)>(s, kb.x, dummy, al[2]);                             \
-          pair_hilo<W, 2 * (MT) + 1>(s, kb.x, dummy, al[3]);                         \
+          pair_hilo<W, 2 * (MT)>(s, kb.x, lane4, dummy, al[2]);                      \
+          pair_hilo<W, 2 * (MT) + 1>(s, kb.x, lane4, dummy, al[3]);                  \
         }                                                                            \
       }                                                                              \
     }                                                                                \
@@ -241,42 +272,121 @@ __device__ __forceinline__ void ktile_step(const DecodeSmem& s, const uint8_t* t
       mma16816(C[MT], al, bq.x, bq.y);                                               \
     }                                                                                \
   }
-  GTQ_MT(0) GTQ_MT(1) GTQ_MT(2) GTQ_MT(3)
+  GTQ_MT(0) GTQ_MT(1)
 #undef GTQ_MT
 }
 
 template <int W, bool SPLIT>
 __device__ __forceinline__ void group_scores(const DecodeSmem& s, const uint8_t* tile, int kt0,
-                                             int kt1, int koff_lane, uint32_t lane_pair, int lane,
-                                             float (&C)[4][4]) {
+                                             int kt1, int koff_lane, uint32_t lane4, int lane,
+                                             float (&C)[2][4]) {
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int r = 0; r < 4; ++r) C[mt][r] = 0.f;
   for (int kt = kt0; kt < kt1; ++kt)
     ktile_step<W, SPLIT>(s, tile, koff_lane + (kt - kt0) * 128 * W, s.meta.kt_nslots[kt] > 4,
-                         lane_pair, s.qf[kt][lane], C);
+                         lane4, s.qf[kt][lane], C);
 }
 
-// P.V for one dim tile: V portion of width VB (32 codes, VB words), 4 token k-tiles
+// P.V for one dim tile and this warp's 32 tokens: 16 codes of width VB per lane
+// (pairs 8h .. 8h + 7 of the lane's 32-code portion), 2 token k-tiles
 template <int VB>
-__device__ __forceinline__ void value_tile(const DecodeSmem& s, const uint32_t* pw,
-                                           uint32_t lane_pair, const uint32_t (&PB)[4][2],
+__device__ __forceinline__ void value_tile(const DecodeSmem& s, const uint8_t* lane_codes, int h,
+                                           uint32_t lane4, const uint32_t (&PB)[2][2],
                                            float (&o)[4]) {
-  uint32_t x[VB + 1];
-#pragma unroll
-  for (int i = 0; i < VB; ++i) x[i] = pw[i];
-  x[VB] = 0u;
+  Bits<16 * VB> v;
+  v.load(lane_codes, 2 * VB * h);
 #define GTQ_V_KTILE(KK)                                                            \
   {                                                                                \
-    const uint32_t av[4] = {pair_hi<VB, 4 * (KK)>(s, x, lane_pair),                \
-                            pair_hi<VB, 4 * (KK) + 1>(s, x, lane_pair),            \
-                            pair_hi<VB, 4 * (KK) + 2>(s, x, lane_pair),            \
-                            pair_hi<VB, 4 * (KK) + 3>(s, x, lane_pair)};           \
+    const uint32_t av[4] = {pair_hi<VB, 4 * (KK)>(s, v.x, lane4),                  \
+                            pair_hi<VB, 4 * (KK) + 1>(s, v.x, lane4),              \
+                            pair_hi<VB, 4 * (KK) + 2>(s, v.x, lane4),              \
+                            pair_hi<VB, 4 * (KK) + 3>(s, v.x, lane4)};             \
     mma16816(o, av, PB[KK][0], PB[KK][1]);                                         \
   }
-  GTQ_V_KTILE(0) GTQ_V_KTILE(1) GTQ_V_KTILE(2) GTQ_V_KTILE(3)
+  GTQ_V_KTILE(0) GTQ_V_KTILE(1)
 #undef GTQ_V_KTILE
+}
+
+// Arrival of this CTA at a merge ticket after its partial is stored: true in
+// every thread of the CTA that arrived last (of `count`); that CTA also resets
+// the ticket for the next call.  The atomic is acquire-release at GPU scope:
+// it publishes this CTA's stores (ordered before it by the CTA barrier) and,
+// in the last arriver, makes the others' stores visible to its loads.
+__device__ bool arrive_last(unsigned* ticket, unsigned count, int* flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned prev;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ticket) : "memory");
+    const int last = prev == count - 1;
+    if (last) asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ticket) : "memory");
+    *flag = last;
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int*>(flag) != 0;
+}
+
+// Merge partials [first, first + count) (count <= kMergeGroup) of the 8 query
+// heads: M = max m_j, L = sum 2^(m_j - M) l_j, o = sum 2^(m_j - M) o_j.  Written
+// as a partial to dst (global) or, normalised (o / L), to o_rot (shared).
+// Thread = (query head, 4 dims, half of the partials); the halves combine by a
+// shuffle.  Partials come from other CTAs: loads bypass L1.
+__device__ void merge_partials(const float* head_parts, int first, int count, float* dst,
+                               float (*o_rot)[kD]) {
+  for (int idx = threadIdx.x; idx < 8 * 32 * 2; idx += blockDim.x) {
+    const int hh = idx >> 6, d4 = (idx >> 1) & 31, sub = idx & 1;
+    float mj[kMergeGroup / 2], lj[kMergeGroup / 2];
+    float4 oj[kMergeGroup / 2];
+#pragma unroll
+    for (int k = 0; k < kMergeGroup / 2; ++k) {
+      const int j = sub + 2 * k;
+      mj[k] = -1e30f;
+      lj[k] = 0.f;
+      oj[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < count) {
+        const float* pj = head_parts + ((size_t)(first + j) * 8 + hh) * kPartialStride;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(pj));
+        mj[k] = ml.x;
+        lj[k] = ml.y;
+        oj[k] = __ldcg(reinterpret_cast<const float4*>(pj + 4) + d4);
+      }
+    }
+    float M = mj[0];
+#pragma unroll
+    for (int k = 1; k < kMergeGroup / 2; ++k) M = fmaxf(M, mj[k]);
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+    float L = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kMergeGroup / 2; ++k) {
+      const float w = exp2f(mj[k] - M);
+      L = fmaf(w, lj[k], L);
+      o.x = fmaf(w, oj[k].x, o.x);
+      o.y = fmaf(w, oj[k].y, o.y);
+      o.z = fmaf(w, oj[k].z, o.z);
+      o.w = fmaf(w, oj[k].w, o.w);
+    }
+    L += __shfl_xor_sync(0xffffffffu, L, 1);
+    o.x += __shfl_xor_sync(0xffffffffu, o.x, 1);
+    o.y += __shfl_xor_sync(0xffffffffu, o.y, 1);
+    o.z += __shfl_xor_sync(0xffffffffu, o.z, 1);
+    o.w += __shfl_xor_sync(0xffffffffu, o.w, 1);
+    if (sub == 0) {
+      if (dst) {
+        float* pd = dst + hh * kPartialStride;
+        reinterpret_cast<float4*>(pd + 4)[d4] = o;
+        if (d4 == 0) {
+          pd[0] = M;
+          pd[1] = L;
+        }
+      } else {
+        const float inv = 1.f / L;
+        *reinterpret_cast<float4*>(&o_rot[hh][4 * d4]) =
+            make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      }
+    }
+  }
 }
 
 template <int VB>
@@ -287,52 +397,62 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
   const int stride = (a.tile_bytes + 127) & ~127;
   const int head = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int nw = blockDim.x >> 5;  // warps in this CTA (<= kWarps)
+  const int nw = blockDim.x >> 5;  // warps in this CTA (even, <= kWarps)
+  const int np = nw >> 1;          // warp pairs: both warps of a pair share one tile
+  const int pair = warp >> 1, wh = warp & 1;  // this warp: tokens 32 wh .. 32 wh + 31
 
+  // Shared memory after DecodeSmem: tile stages, stage-major (stage st of pair
+  // p at (st * np + p) * stride); at setup the transposed key rotation M_h^T
+  // and the rotation's partial sums sit at a.rot_off, inside stages >= 1, whose
+  // tiles load once the rotation is done.
+  const int stages = a.stages;
+  uint8_t* stage_base = smem_raw + stage_off;
+  auto stage_ptr = [&](int st) { return stage_base + (size_t)(st * np + pair) * stride; };
+  float* mt = reinterpret_cast<float*>(stage_base + a.rot_off);  // M_h^T [dim][pos]
+  float* rot_part = mt + kD * kD;                                 // [4][8][128]
+  float(*qt)[8] = reinterpret_cast<float(*)[8]>(&s.qs[0][0]);    // q^T [dim][head]
+
+  // Setup: lookup tables, head metadata and M_h^T by bulk copies (issued
+  // first: nothing here depends on the previous grid), then stage 0 of every
+  // pair; the queries follow the grid-dependency wait.
   if (tid == 0) {
-    s.meta = a.meta[head];
-    for (int w = 0; w < nw; ++w)
-      for (int st = 0; st < kStages; ++st) mbar_init(&s.bar[w][st], 1);
+    mbar_init(&s.setup_bar, 1);
+    for (int p = 0; p < np; ++p)
+      for (int st = 0; st < stages; ++st) {
+        mbar_init(&s.bar[p][st], 1);
+        s.done[p][st] = 0u;
+      }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&s.setup_bar)),
+                 "r"((unsigned)(kDecodeImageBytes + sizeof(HeadMeta) + kD * kD * sizeof(float)))
+                 : "memory");
+    bulk_copy(s.tab, a.dec_image, kDecodeImageBytes, &s.setup_bar);
+    bulk_copy(&s.meta, a.meta + head, sizeof(HeadMeta), &s.setup_bar);
+    bulk_copy(mt, a.mrow_t + (size_t)head * kD * kD, kD * kD * sizeof(float), &s.setup_bar);
   }
-  // lookup tables: one 16-byte-vector copy of the prebuilt image
-  static_assert(offsetof(DecodeSmem, single) == kPairBytes, "image layout");
-  for (int i = tid; i < kDecodeImageBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(s.pair)[i] = a.dec_image[i];
-  __syncthreads();
+  __syncthreads();  // barrier initialisation visible
   pdl_launch_dependents();
+  bool failed = __syncthreads_or(!mbar_wait(&s.setup_bar, 0));
   const HeadMeta& m = s.meta;
   const int load_bytes = 1024 * (a.kb + VB) + 128 + 128 * m.n_groups;
   const int knorm_off = 1024 * (a.kb + VB) + 128, vnorm_off = 1024 * (a.kb + VB);
-  uint32_t lane_pair[4];
-#pragma unroll
-  for (int w = 0; w < 4; ++w) lane_pair[w] = kPairOff(w) | (uint32_t)(lane * 4);
+  const uint32_t lane4 = (uint32_t)lane << 2;
 
-  // tiles of this split, dealt to warps round-robin; the packed cache does not
-  // depend on the previous grid, so its first tiles load before the wait
+  // tiles of this split, dealt to warp pairs round-robin
   const int64_t per = (a.tiles_T + a.splits - 1) / a.splits;
-  const int64_t tb0 = (int64_t)split * per, tb1 = min(a.tiles_T, tb0 + per);
+  const int64_t tb0 = (int64_t)split * per, tb1 = failed ? tb0 : min(a.tiles_T, tb0 + per);
   const uint8_t* head_base = a.packed + (size_t)head * a.n_tiles * a.tile_bytes;
-  uint8_t* my_stage0 = smem_raw + stage_off + (size_t)(warp * kStages) * stride;
-  if (lane == 0) {
-    for (int st = 0; st < kStages; ++st) {
-      const int64_t tile = tb0 + warp + (int64_t)nw * st;
-      if (tile < tb1)
-        bulk_load(my_stage0 + (size_t)st * stride, head_base + (size_t)tile * a.tile_bytes,
-                  (unsigned)load_bytes, &s.bar[warp][st]);
+  const uint64_t stream_pol = evict_first_policy();
+  auto first_loads = [&](int st0, int st1) {
+    if (wh == 0 && lane == 0 && !failed) {
+      for (int st = st0; st < st1; ++st) {
+        const int64_t tile = tb0 + pair + (int64_t)np * st;
+        if (tile < tb1) tile_load(stage_ptr(st), head_base + (size_t)tile * a.tile_bytes,
+                                  (unsigned)load_bytes, &s.bar[pair][st], stream_pol);
+      }
     }
-  }
-  // M_h rows of this thread's first rotation task (pos, half of d), prefetched
-  // before the wait: they do not depend on the previous grid
-  const int rot_pos = tid & (kD - 1), rot_half = (tid >> 7) & 1;
-  const bool rot_live = tid < 2 * kD && (rot_pos >> 1) < m.n_slots;
-  float4 mv[16];
-  if (rot_live) {
-    const float4* row = reinterpret_cast<const float4*>(
-        a.mrow + ((size_t)head * kD + rot_pos) * kD + 64 * rot_half);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) mv[j] = row[j];
-  }
+  };
+  first_loads(0, 1);
   pdl_wait();  // the queries may come from the previous grid
   {
     const int b = head / a.hkv, h = head % a.hkv;
@@ -344,53 +464,47 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
         v = a.q_fp32 ? reinterpret_cast<const float*>(a.q)[qi]
                      : __half2float(reinterpret_cast<const __half*>(a.q)[qi]);
       }
-      s.qs[hh][d] = v;
+      qt[d][hh] = v;
     }
   }
   __syncthreads();
   // q_rot[hh][pos] = M_h[pos] . q[hh] * log2(e) / (sqrt(d) sqrt(m_g)).  Task = (pos,
-  // half of d): 16 float4 of the row, 8 query heads; partial sums in s.qf.
-  {
-    static_assert(sizeof(DecodeSmem::qf) >= 2 * 8 * kD * sizeof(float), "rotation scratch");
-    float* part = reinterpret_cast<float*>(s.qf);  // [2][8][128] partial dot products
-    for (int task = tid; task < 2 * kD; task += blockDim.x) {
-      const int pos = task & (kD - 1), qd = task >> 7;
-      const bool live = (pos >> 1) < m.n_slots;
-      if (task != tid && live) {  // later tasks of a small CTA: load now
-        const float4* row =
-            reinterpret_cast<const float4*>(a.mrow + ((size_t)head * kD + pos) * kD + 64 * qd);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) mv[j] = row[j];
-      }
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (live) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int d = 64 * qd + 4 * j;
-#pragma unroll
-          for (int hh = 0; hh < 8; ++hh) {
-            const float4 qv = *reinterpret_cast<const float4*>(&s.qs[hh][d]);
-            acc[hh] = fmaf(mv[j].x, qv.x, acc[hh]);
-            acc[hh] = fmaf(mv[j].y, qv.y, acc[hh]);
-            acc[hh] = fmaf(mv[j].z, qv.z, acc[hh]);
-            acc[hh] = fmaf(mv[j].w, qv.w, acc[hh]);
-          }
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < 8; ++hh) part[(qd * 8 + hh) * kD + pos] = acc[hh];
+  // quarter of d): a warp holds 32 consecutive positions of one quarter, so the
+  // M_h^T reads are contiguous and the q reads broadcasts.
+  for (int task = tid; task < 4 * kD; task += blockDim.x) {
+    const int pos = task & (kD - 1), qd = task >> 7;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int i = 0; i < 32; ++i) {
+      const int d = 32 * qd + i;
+      const float mv = mt[d * kD + pos];
+      const float4 qa = *reinterpret_cast<const float4*>(&qt[d][0]);
+      const float4 qb = *reinterpret_cast<const float4*>(&qt[d][4]);
+      acc[0] = fmaf(mv, qa.x, acc[0]);
+      acc[1] = fmaf(mv, qa.y, acc[1]);
+      acc[2] = fmaf(mv, qa.z, acc[2]);
+      acc[3] = fmaf(mv, qa.w, acc[3]);
+      acc[4] = fmaf(mv, qb.x, acc[4]);
+      acc[5] = fmaf(mv, qb.y, acc[5]);
+      acc[6] = fmaf(mv, qb.z, acc[6]);
+      acc[7] = fmaf(mv, qb.w, acc[7]);
     }
-    __syncthreads();
-    for (int i = tid; i < 8 * kD; i += blockDim.x) {
-      const int hh = i >> 7, pos = i & (kD - 1), slot = pos >> 1;
-      // base-2 logits: log2(e) / sqrt(128), and 1/sqrt(m_g) of the group
-      const float sc = slot < m.n_slots ? m.inv_sqrt_m[m.slot_group[slot]] *
-                                              (1.4426950408889634f * 0.08838834764831845f)
-                                        : 0.f;
-      s.qr[hh][pos] = (part[(0 * 8 + hh) * kD + pos] + part[(1 * 8 + hh) * kD + pos]) * sc;
-    }
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) rot_part[(qd * 8 + hh) * kD + pos] = acc[hh];
   }
   __syncthreads();
+  for (int i = tid; i < 8 * kD; i += blockDim.x) {
+    const int hh = i >> 7, pos = i & (kD - 1), slot = pos >> 1;
+    // base-2 logits: log2(e) / sqrt(128), and 1/sqrt(m_g) of the group
+    const float sc = slot < m.n_slots ? m.inv_sqrt_m[m.slot_group[slot]] *
+                                            (1.4426950408889634f * 0.08838834764831845f)
+                                      : 0.f;
+    s.qr[hh][pos] = ((rot_part[hh * kD + pos] + rot_part[(8 + hh) * kD + pos]) +
+                     (rot_part[(16 + hh) * kD + pos] + rot_part[(24 + hh) * kD + pos])) * sc;
+  }
+  __syncthreads();  // M_h^T and the partial sums are dead: stages >= 1 may load
+  if (wh == 0 && lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  first_loads(1, stages);
   // B fragments (query) of every decode k-tile; slots past the k-tile's run are zero
   for (int idx = tid; idx < m.n_ktiles * 32; idx += blockDim.x) {
     const int kt = idx >> 5, ln = idx & 31, gg = ln >> 2, tt = ln & 3;
@@ -413,47 +527,45 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
   float O[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
-  bool failed = false;
 
-  int it = 0;
-  for (int64_t tile = tb0 + warp; tile < tb1; tile += nw, ++it) {
-    const int st = it % kStages;
-    const unsigned phase = (unsigned)(it / kStages) & 1u;
-    if (!mbar_wait(&s.bar[warp][st], phase)) {
+  int it = 0, st = 0;
+  unsigned phase = 0u;
+  for (int64_t tile = tb0 + pair; tile < tb1; tile += np, ++it) {
+    if (!mbar_wait(&s.bar[pair][st], phase)) {
       failed = true;
       break;
     }
-    const uint8_t* tl = my_stage0 + (size_t)st * stride;
-    const uint32_t* tl32 = reinterpret_cast<const uint32_t*>(tl);
+    const uint8_t* tl = stage_ptr(st);
 
     // ------------------------------------------------------------ scores
-    float S[4][4], C[4][4];
+    float S[2][4], C[2][4];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int r = 0; r < 4; ++r) S[mt][r] = 0.f;
     for (int gi = 0; gi < m.n_groups; ++gi) {
       const int W = m.grp_width[gi], split = m.grp_split[gi];
       const int kt0 = m.grp_kt0[gi], kt1 = m.grp_kt1[gi];
-      const int koff_lane = m.slot_koff[m.grp_first_slot[gi]] + 16 * W * t + 2 * W * g;
+      // lane portion of slot t: 16W bits at byte 16W t + 2W g; this warp's half: + W wh
+      const int koff_lane = m.slot_koff[m.grp_first_slot[gi]] + W * (16 * t + 2 * g + wh);
       switch (2 * W + split) {
-#define GTQ_GROUP(WW)                                                                        \
-  case 2 * WW:                                                                               \
-    group_scores<WW, false>(s, tl, kt0, kt1, koff_lane, lane_pair[WW < 4 ? WW : 0], lane, C); \
-    break;                                                                                   \
-  case 2 * WW + 1:                                                                           \
-    group_scores<WW, true>(s, tl, kt0, kt1, koff_lane, lane_pair[WW < 4 ? WW : 0], lane, C); \
+#define GTQ_GROUP(WW)                                                        \
+  case 2 * WW:                                                               \
+    group_scores<WW, false>(s, tl, kt0, kt1, koff_lane, lane4, lane, C);     \
+    break;                                                                   \
+  case 2 * WW + 1:                                                           \
+    group_scores<WW, true>(s, tl, kt0, kt1, koff_lane, lane4, lane, C);      \
     break;
         GTQ_GROUP(1) GTQ_GROUP(2) GTQ_GROUP(3) GTQ_GROUP(4)
         GTQ_GROUP(5) GTQ_GROUP(6) GTQ_GROUP(7) GTQ_GROUP(8)
 #undef GTQ_GROUP
         default: break;
       }
-      // group complete: scale by its fp16 norms
-      const uint4 nq = *reinterpret_cast<const uint4*>(tl + knorm_off + gi * 128 + g * 16);
+      // group complete: scale by its fp16 norms (tokens g + 8u, u = 4wh .. 4wh + 3)
+      const uint2 nq = *reinterpret_cast<const uint2*>(tl + knorm_off + gi * 128 + g * 16 + wh * 8);
       const __half2* nh = reinterpret_cast<const __half2*>(&nq);
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
+      for (int mt = 0; mt < 2; ++mt) {
         const float2 n = __half22float2(nh[mt]);
         S[mt][0] = fmaf(n.x, C[mt][0], S[mt][0]);
         S[mt][1] = fmaf(n.x, C[mt][1], S[mt][1]);
@@ -462,11 +574,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
       }
     }
     // ------------------------------------------------------ online softmax
-    const int64_t tok0 = tile * kTile;
-    const bool full = tok0 + kTile <= a.T;
+    const int64_t tok0 = tile * kTile + 32 * wh;
+    const bool full = tok0 + 32 <= a.T;
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int j = 16 * mt + g + 8 * (r >> 1);
@@ -474,18 +586,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
         mx[r & 1] = fmaxf(mx[r & 1], S[mt][r]);
       }
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 4));
-      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 8));
-      mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 16));
+    for (int q2 = 0; q2 < 2; ++q2) {
+      mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], 4));
+      mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], 8));
+      mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], 16));
     }
     float alpha[2];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const float mn = fmaxf(mrun[hh], mx[hh]);
-      alpha[hh] = exp2f(mrun[hh] - mn);
-      mrun[hh] = mn;
-      lrun[hh] *= alpha[hh];
+    for (int q2 = 0; q2 < 2; ++q2) {
+      const float mn = fmaxf(mrun[q2], mx[q2]);
+      alpha[q2] = exp2f(mrun[q2] - mn);
+      mrun[q2] = mn;
+      lrun[q2] *= alpha[q2];
     }
     if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
@@ -496,12 +608,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
         O[i][3] *= alpha[1];
       }
     }
-    const uint4 vq = *reinterpret_cast<const uint4*>(tl + vnorm_off + g * 16);
+    const uint2 vq = *reinterpret_cast<const uint2*>(tl + vnorm_off + g * 16 + wh * 8);
     const __half2* vnh = reinterpret_cast<const __half2*>(&vq);
-    uint32_t PB[4][2];
+    uint32_t PB[2][2];
     const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128)
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
+    for (int mt = 0; mt < 2; ++mt) {
       float2 vn = __half22float2(vnh[mt]);
       vn.x *= inv_sqrt_d;
       vn.y *= inv_sqrt_d;
@@ -518,32 +630,52 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
       PB[mt][1] = movmatrix_t(pack_half2(__float2half_rn(pp[2]), __float2half_rn(pp[3])));
     }
     // ---------------------------------------------------------------- P.V
-    const uint32_t* vcodes = tl32 + 256 * a.kb;
+    const uint8_t* vcodes = tl + 1024 * a.kb;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      value_tile<VB>(s, vcodes + ((i * 8 + g) * 4 + t) * VB, lane_pair[VB < 4 ? VB : 0], PB, O[i]);
-    // -------------------------------------------------- refill this stage
+      value_tile<VB>(s, vcodes + ((i * 8 + g) * 4 + t) * VB * 4, wh, lane4, PB, O[i]);
+    // ------------------------------------- release the stage; the second warp
+    // of the pair to release it refills it
     __syncwarp();
     if (lane == 0) {
-      const int64_t nxt = tile + (int64_t)nw * kStages;
-      if (nxt < tb1) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        bulk_load(my_stage0 + (size_t)st * stride, head_base + (size_t)nxt * a.tile_bytes,
-                  (unsigned)load_bytes, &s.bar[warp][st]);
+      __threadfence_block();
+      const unsigned prev = atomicAdd(&s.done[pair][st], 1u);
+      if (prev & 1u) {
+        __threadfence_block();
+        const int64_t nxt = tile + (int64_t)np * stages;
+        if (nxt < tb1) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          tile_load(stage_ptr(st), head_base + (size_t)nxt * a.tile_bytes, (unsigned)load_bytes,
+                    &s.bar[pair][st], stream_pol);
+        }
       }
+    }
+    if (++st == stages) {
+      st = 0;
+      phase ^= 1u;
     }
   }
   if (failed && lane == 0) atomicOr(a.status, kStatusTimeout);
 
-  // --------------------------------------------- merge the 4 warps in the CTA
+  // ------------------------------------------------- merge the warps in the CTA
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     lrun[hh] += __shfl_xor_sync(0xffffffffu, lrun[hh], 4);
     lrun[hh] += __shfl_xor_sync(0xffffffffu, lrun[hh], 8);
     lrun[hh] += __shfl_xor_sync(0xffffffffu, lrun[hh], 16);
   }
-  __syncthreads();  // every warp is done with its stages: reuse them for o
-  float* wo = reinterpret_cast<float*>(smem_raw + stage_off);  // [warp][8 heads][128]
+  __syncthreads();  // every warp is done with its stages: reuse them for R_V and o
+  // R_V is staged in every CTA (only the one that finishes the merge uses it;
+  // the copy is in flight meanwhile, and every CTA waits for it before exit)
+  float* rv = reinterpret_cast<float*>(stage_base);            // R_V [128][128]
+  float* wo = reinterpret_cast<float*>(stage_base) + kD * kD;  // [warp][8][128]
+  if (tid == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&s.setup_bar)),
+                 "r"((unsigned)(kD * kD * sizeof(float)))
+                 : "memory");
+    bulk_copy(rv, a.rot_v, kD * kD * sizeof(float), &s.setup_bar);
+  }
   if (g == 0) {
     s.wm[warp][2 * t] = mrun[0];
     s.wm[warp][2 * t + 1] = mrun[1];
@@ -573,124 +705,71 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
     s.hl[hh] = L;
   }
   __syncthreads();
+  const int S = a.splits;
   float* head_parts = a.partials + (size_t)head * kPartialSlots * 8 * kPartialStride;
   float* part = head_parts + (size_t)split * 8 * kPartialStride;
-  for (int idx = tid; idx < 8 * kPartialStride; idx += blockDim.x) {
-    const int hh = idx / kPartialStride, k = idx % kPartialStride;
-    float v;
-    if (k == 0) {
-      v = s.hm[hh];
-    } else if (k == 1) {
-      v = s.hl[hh];
+  // this CTA's (m, l, o_rot): the output itself with a single split, else its
+  // partial in global memory
+  for (int idx = tid; idx < 8 * kD; idx += blockDim.x) {
+    const int hh = idx >> 7, d = idx & (kD - 1);
+    float v = 0.f;
+    for (int w = 0; w < nw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * 8 + hh) * kD + d], v);
+    if (S == 1) {
+      s.qs[hh][d] = v / s.hl[hh];
     } else {
-      v = 0.f;
-      for (int w = 0; w < nw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * 8 + hh) * kD + k - 2], v);
+      part[hh * kPartialStride + 4 + d] = v;
+      if (d == 0) *reinterpret_cast<float2*>(part + hh * kPartialStride) = make_float2(s.hm[hh], s.hl[hh]);
     }
-    part[idx] = v;
   }
-  // ---------------- merge of the splits.  Every CTA of the head arrives at a
-  // per-head barrier (arrival count + generation, bounded spin) once its partial
-  // is in global memory; all CTAs of the head are resident (one wave).  Then
-  // this CTA merges the outputs it owns: query heads split, split + S, ... when
-  // S < G_q; otherwise query head split % G_q and its output dims d with
-  // d % nc == split / G_q (nc = CTAs sharing that query head).
-  const int S = a.splits, G = a.gq;
-  if (S > 1) {
-    __syncthreads();
-    if (tid == 0) {
-      unsigned* bar = a.tickets + (size_t)head * 2;  // [0] arrivals, [1] generation
-      const unsigned gen0 = *reinterpret_cast<volatile unsigned*>(&bar[1]);
-      __threadfence();
-      if (atomicAdd(&bar[0], 1u) == (unsigned)(S - 1)) {
-        bar[0] = 0u;
-        __threadfence();
-        atomicExch(&bar[1], gen0 + 1u);
+  // ---------------- merge of the splits, without waiting: the last CTA to
+  // arrive in a group of kMergeGroup splits merges the group into a
+  // second-level partial, and the last group to finish merges those.  Arrival
+  // order comes from per-head tickets (acquire-release atomics); the last
+  // arriver resets its ticket for the next call.
+  bool finish = S == 1;
+  if (!finish) {
+    unsigned* tickets = a.tickets + (size_t)head * (1 + kMaxMergeGroups);
+    const int n_groups = (S + kMergeGroup - 1) / kMergeGroup;
+    const int grp = split / kMergeGroup;
+    const int n1 = min(kMergeGroup, S - grp * kMergeGroup);
+    if (arrive_last(&tickets[1 + grp], (unsigned)n1, &s.flag)) {
+      if (n_groups == 1) {
+        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qs);
+        finish = true;
       } else {
-        unsigned spins = 0;
-        while (*reinterpret_cast<volatile unsigned*>(&bar[1]) == gen0) {
-          if (++spins > kBarrierSpinLimit) {
-            atomicOr(a.status, kStatusTimeout);
-            break;
-          }
-          __nanosleep(64);
+        merge_partials(head_parts, grp * kMergeGroup, n1,
+                       head_parts + (size_t)(kMaxSplits + grp) * 8 * kPartialStride, nullptr);
+        if (arrive_last(&tickets[0], (unsigned)n_groups, &s.flag)) {
+          merge_partials(head_parts, kMaxSplits, n_groups, nullptr, s.qs);
+          finish = true;
         }
       }
-      __threadfence();
     }
-    __syncthreads();
   }
-  __syncthreads();  // wo (stage area) fully read before the scratch below reuses it
-  float* rot = reinterpret_cast<float*>(smem_raw + stage_off);  // scratch: stages are idle
-  const int P = max(1, (int)blockDim.x / kD);                   // threads per output dim
-  const int b = head / a.hkv, h = head % a.hkv;
-  const int hh0 = S < G ? split : split % G, hh_step = S < G ? S : G;
-  const int nc = S < G ? 1 : (S - split % G + G - 1) / G, c = S < G ? 0 : split / G;
-  for (int hh = hh0; hh < G; hh += hh_step) {
-    // merged o_rot[hh][:]: P threads per dim, each over splits j = p, p + P, ...
-    for (int idx = tid; idx < P * kD; idx += blockDim.x) {
-      const int p = idx / kD, d = idx % kD;
-      const float* q = head_parts + hh * kPartialStride;
-      float M = -1e30f, L = 0.f, o = 0.f;
-      for (int j0 = p; j0 < S; j0 += 16 * P) {
-        float vm[16], vl[16], vo[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int j = j0 + k * P;
-          const bool in = j < S;
-          const float* pj = q + (size_t)j * 8 * kPartialStride;
-          vm[k] = in ? __ldcg(pj) : -1e30f;
-          vl[k] = in ? __ldcg(pj + 1) : 0.f;
-          vo[k] = in ? __ldcg(pj + 2 + d) : 0.f;
-        }
-        float mc = vm[0];
-#pragma unroll
-        for (int k = 1; k < 16; ++k) mc = fmaxf(mc, vm[k]);
-        const float mn = fmaxf(M, mc), sc = exp2f(M - mn);
-        L *= sc;
-        o *= sc;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float w = exp2f(vm[k] - mn);
-          L = fmaf(w, vl[k], L);
-          o = fmaf(w, vo[k], o);
-        }
-        M = mn;
+  const bool rv_ok = mbar_wait(&s.setup_bar, 1);  // no CTA exits with the copy in flight
+  if (!finish) return;
+  if (!rv_ok) {
+    if (tid == 0) atomicOr(a.status, kStatusTimeout);
+    return;
+  }
+  __syncthreads();
+  // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r]
+  {
+    const int b = head / a.hkv, h = head % a.hkv;
+    float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
+    for (int idx = tid; idx < 8 * (kD / 2); idx += blockDim.x) {
+      const int hh = idx / (kD / 2), dd = 2 * (idx % (kD / 2));
+      if (hh >= a.gq) continue;
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < kD; ++r) {
+        const float2 w = *reinterpret_cast<const float2*>(rv + r * kD + dd);
+        const float o = s.qs[hh][r];
+        acc0 = fmaf(w.x, o, acc0);
+        acc1 = fmaf(w.y, o, acc1);
       }
-      rot[(p * 3 + 0) * kD + d] = M;
-      rot[(p * 3 + 1) * kD + d] = L;
-      rot[(p * 3 + 2) * kD + d] = o;
+      *reinterpret_cast<float2*>(out_head + hh * kD + dd) = make_float2(acc0, acc1);
     }
-    __syncthreads();
-    for (int d = tid; d < kD; d += blockDim.x) {
-      float M = -1e30f;
-      for (int p = 0; p < P; ++p) M = fmaxf(M, rot[(p * 3) * kD + d]);
-      float L = 0.f, o = 0.f;
-      for (int p = 0; p < P; ++p) {
-        const float w = exp2f(rot[(p * 3) * kD + d] - M);
-        L = fmaf(w, rot[(p * 3 + 1) * kD + d], L);
-        o = fmaf(w, rot[(p * 3 + 2) * kD + d], o);
-      }
-      s.qs[0][d] = o / L;  // o_rot[hh][d]
-    }
-    __syncthreads();
-    // out[dd] = sum_r R_V[r][dd] o_rot[r] for this CTA's dims dd = c, c + nc, ...:
-    // 16 lanes per dim, 8 rows each
-    const int n_dims = (kD - c + nc - 1) / nc;
-    const int n_items = ((n_dims * 16 + 31) / 32) * 32;  // whole warps: the shuffles need every lane
-    for (int idx = tid; idx < n_items; idx += blockDim.x) {
-      const bool valid = idx < n_dims * 16;
-      const int dd = c + (idx >> 4) * nc, r0 = (idx & 15) * 8;
-      float acc = 0.f;
-      if (valid) {
-#pragma unroll
-        for (int r = r0; r < r0 + 8; ++r) acc = fmaf(__ldg(a.rot_v + r * kD + dd), s.qs[0][r], acc);
-      }
-#pragma unroll
-      for (int o = 8; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, 16);
-      if (valid && (idx & 15) == 0)
-        a.out[((size_t)b * a.hkv * a.gq + (size_t)h * a.gq + hh) * kD + dd] = acc;
-    }
-    __syncthreads();
   }
 }
 
@@ -720,7 +799,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.meta = p->d_meta;
   a.q = q;
   a.q_fp32 = q_dtype == GTQ_DTYPE_FP32;
-  a.mrow = p->d_mrow;
+  a.mrow_t = p->d_mrow_t;
   a.rot_v = p->tab.rot_v;
   a.out = out;
   a.tickets = p->d_tickets;
@@ -739,11 +818,24 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   const size_t stride = (p->tile_bytes + 127) & ~size_t(127);
   int dev_smem = 0;
   cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
-  int nw = (int)std::min<size_t>(kWarps, (dev_smem - stage_off) / (stride * kStages));
-  nw = std::max(nw, 1);
-  // stages; reused at the end for the warps' o (nw x 4 KB) and R_V (128 x 129 floats)
-  const size_t smem = stage_off + std::max({stride * nw * kStages, (size_t)nw * 8 * kD * 4,
-                                            (size_t)kD * (kD + 1) * 4});
+  // Stage area: the tile stages; at the end R_V and the warps' o; at setup,
+  // the setup scratch (M_h^T and the rotation's partial sums) at its top, clear
+  // of stage 0.  Three stages per pair when all pairs fit with them, else two,
+  // with as many pairs as fit.
+  constexpr size_t kSetupScratch = (size_t)kD * kD * 4 + (size_t)4 * 8 * kD * 4;
+  auto area_for = [&](int np_, int st_) {
+    return std::max({stride * np_ * st_, (size_t)kD * kD * 4 + (size_t)2 * np_ * 8 * kD * 4,
+                     stride * np_ + kSetupScratch});
+  };
+  int stages = kMaxStages, np = kPairs;
+  if (stage_off + area_for(np, stages) > (size_t)dev_smem) stages = 2;
+  while (np > 1 && stage_off + area_for(np, stages) > (size_t)dev_smem) --np;
+  if (stage_off + area_for(np, stages) > (size_t)dev_smem) return cudaErrorInvalidValue;
+  a.stages = stages;
+  const int nw = 2 * np;
+  const size_t area = area_for(np, stages);
+  a.rot_off = (int)(area - kSetupScratch);
+  const size_t smem = stage_off + area;
   int per_sm = 1;
   switch (a.vb) {
 #define GTQ_OCC_VB(VB)                                                                           \
@@ -758,7 +850,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   // one wave of resident CTAs: the split merge waits for every CTA of a head
   const int capacity = std::max(1, per_sm) * p->n_sms;
   int splits = std::max(1, capacity / p->n_heads);
-  splits = (int)std::min<int64_t>(splits, (a.tiles_T + nw - 1) / nw);
+  splits = (int)std::min<int64_t>(splits, (a.tiles_T + np - 1) / np);
   splits = std::max(1, std::min(splits, kMaxSplits));
   // every split must own at least one tile
   const int64_t per = (a.tiles_T + splits - 1) / splits;

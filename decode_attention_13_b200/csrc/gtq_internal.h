@@ -18,7 +18,7 @@ constexpr int kMaxGq = 8;               // query heads per KV head handled by de
 constexpr int kLutEntries = 510;        // sum over w = 1..8 of 2^w
 constexpr int kThrEntries = 502;        // sum over w = 1..8 of (2^w - 1)
 constexpr int kMaxSplits = 256;         // context splits per head in decode
-constexpr int kPartialStride = 2 + kD;  // (m, l, o[128]) per (split, q head)
+constexpr int kPartialStride = 4 + kD;  // (m, l, -, -, o[128]) per (split, q head)
 constexpr int kMergeGroup = 16;          // splits merged together at the first merge level
 constexpr int kMaxMergeGroups = kMaxSplits / kMergeGroup;
 constexpr int kPartialSlots = kMaxSplits + kMaxMergeGroups;  // per head: level 1 + level 2
@@ -53,17 +53,35 @@ struct HeadMeta {
   uint8_t kt_flags[kMaxKt];       // bit 0: first k-tile of its group, bit 1: last
 };
 
-// Decode lookup tables, laid out exactly as the decode kernel's shared memory:
-// pair tables (widths 1..3, fp16 half2 (cb[c0], cb[c1]) at entry c0 | c1 << w,
-// one copy per lane: word offset kPairOff(w)/4 + entry * 32 + lane), then
-// single-code tables (widths 1..8, word kSingleOff(w)/4 + code = fp16 hi part in
-// the low half, fp16 lo part in the high half).  The offsets make
-// "offset | index" an address without an add.
-constexpr int kPairBytes = 10752;
-constexpr int kSingleBytes = 2048;
-constexpr int kDecodeImageBytes = kPairBytes + kSingleBytes;
+// Decode lookup tables, laid out exactly as the decode kernel's shared memory.
+// Every table is addressed as "region offset + index", where the index is built
+// by one shift and one mask-or from the packed bits:
+//  * pair tables, widths 1..3: entry c0 | c1 << w holds the fp16 half2
+//    (cb[c0], cb[c1]) (hi parts); one copy per lane, at byte
+//    kPairOff(w) + entry * 128 + lane * 4, so a warp-wide lookup never has a
+//    bank conflict;
+//  * lane-private single-code tables, widths 4..6: entry c holds fp16 hi part
+//    (low half) and lo part (high half) of cb[c], at byte
+//    kLaneSingleOff(w) + c * 128 + lane * 4;
+//  * shared single-code tables, widths 1..8 (same entry format), at byte
+//    kSharedSingles + kSingleOff(w) + c * 4 (one copy; used for the lo parts of
+//    narrow split groups and for widths 7 and 8).
+constexpr int kDecodeImageBytes = 28672;
 __host__ __device__ constexpr uint32_t kPairOff(int w) { return w == 3 ? 0u : (w == 2 ? 8192u : 10240u); }
+__host__ __device__ constexpr uint32_t kLaneSingleOff(int w) {
+  return w == 4 ? 12288u : (w == 5 ? 24576u : 16384u);
+}
+constexpr uint32_t kSharedSingles = 14336;
 __host__ __device__ constexpr uint32_t kSingleOff(int w) { return 2048u - (8u << w); }
+// regions: pairs w3 [0, 8K), w2 [8K, 10K), w1 [10K, 10.5K); lane singles w4
+// [12K, 14K), w6 [16K, 24K), w5 [24K, 28K); shared singles [14K, 16K)
+static_assert(kPairOff(2) >= kPairOff(3) + (64u << 7) && kPairOff(1) >= kPairOff(2) + (16u << 7) &&
+                  kLaneSingleOff(4) >= kPairOff(1) + (4u << 7) &&
+                  kSharedSingles >= kLaneSingleOff(4) + (16u << 7) &&
+                  kLaneSingleOff(6) >= kSharedSingles + 2048u &&
+                  kLaneSingleOff(5) >= kLaneSingleOff(6) + (64u << 7) &&
+                  (uint32_t)kDecodeImageBytes >= kLaneSingleOff(5) + (32u << 7),
+              "decode table regions overlap");
 
 // Code lookup table of the tensor-core quantizer, one part per width w = 1..8.
 // Cell of an fp32 value z: floor(z * inv[w]) + k[w], evaluated as
@@ -123,6 +141,7 @@ struct gtq_plan {
   uint8_t* d_bits;    // [heads][n_blocks]
   gtq::HeadMeta* d_meta;  // [heads]
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
+  float* d_mrow_t;    // [heads][128][128] the same, transposed: [dim][packed position]
   uint8_t* d_bimg;    // [heads] M_h as the quantizer's tensor-core B operand (64 KB each)
   float* d_qrot;      // [heads][8][128] rotated, scaled queries (decode workspace)
   float* d_partials;  // [heads][kPartialSlots][8][kPartialStride]
