@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kPairs = 8;  // one CTA per SM: up to 8 warp pairs, 2 tile stages per pair
 constexpr int kWarps = 2 * kPairs;
-constexpr int kMaxStages = 3;  // tile stages per warp pair (3 when 8 pairs fit, else 2)
+constexpr int kMaxStages = 2;  // tile stages per warp pair
 constexpr unsigned kSpinLimit = 1u << 26;
 
 struct DecodeArgs {
@@ -39,7 +39,7 @@ struct DecodeArgs {
   float* out;           // [B][Hq][128]
   const uint4* dec_image;  // lookup tables (kDecodeImageBytes)
   float* partials;      // [heads][kPartialSlots][8][kPartialStride]
-  unsigned* tickets;    // [heads][1 + kMaxMergeGroups]
+  unsigned* tickets;    // [heads][1 + kMaxMergeGroups] arrival counters of the split merge
   int* status;
   int q_fp32;
   int hkv, gq;
@@ -143,6 +143,7 @@ struct DecodeSmem {
   uint32_t tab[kDecodeImageBytes / 4];
   uint4 qf[kMaxKt][32];  // per k-tile & lane: hi(slot A), hi(slot B), lo(A), lo(B)
   alignas(16) HeadMeta meta;
+  uint2 gdesc[kMaxGroups];  // per key group: 2 width + split | kt0 << 8 | kt1 << 16; byte offset
   uint64_t setup_bar;              // lookup tables and metadata loaded
   uint64_t bar[kPairs][kMaxStages];   // tile loaded (bulk copy complete)
   unsigned done[kPairs][kMaxStages];  // releases of a stage by the two warps of its pair
@@ -277,13 +278,15 @@ __device__ __forceinline__ void ktile_step(const DecodeSmem& s, const uint8_t* t
 }
 
 template <int W, bool SPLIT>
-__device__ __forceinline__ void group_scores(const DecodeSmem& s, const uint8_t* tile, int kt0,
-                                             int kt1, int koff_lane, uint32_t lane4, int lane,
+__device__ __forceinline__ void group_scores(const DecodeSmem& s, const uint8_t* tile, uint2 desc,
+                                             int koff_lane, uint32_t lane4, int lane,
                                              float (&C)[2][4]) {
+  const int kt0 = (desc.x >> 8) & 0xff, kt1 = (desc.x >> 16) & 0xff;
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int r = 0; r < 4; ++r) C[mt][r] = 0.f;
+#pragma unroll 1
   for (int kt = kt0; kt < kt1; ++kt)
     ktile_step<W, SPLIT>(s, tile, koff_lane + (kt - kt0) * 128 * W, s.meta.kt_nslots[kt] > 4,
                          lane4, s.qf[kt][lane], C);
@@ -330,61 +333,65 @@ __device__ bool arrive_last(unsigned* ticket, unsigned count, int* flag) {
 // Merge partials [first, first + count) (count <= kMergeGroup) of the 8 query
 // heads: M = max m_j, L = sum 2^(m_j - M) l_j, o = sum 2^(m_j - M) o_j.  Written
 // as a partial to dst (global) or, normalised (o / L), to o_rot (shared).
-// Thread = (query head, 4 dims, half of the partials); the halves combine by a
-// shuffle.  Partials come from other CTAs: loads bypass L1.
-__device__ void merge_partials(const float* head_parts, int first, int count, float* dst,
-                               float (*o_rot)[kD]) {
-  for (int idx = threadIdx.x; idx < 8 * 32 * 2; idx += blockDim.x) {
-    const int hh = idx >> 6, d4 = (idx >> 1) & 31, sub = idx & 1;
-    float mj[kMergeGroup / 2], lj[kMergeGroup / 2];
+// Work item = (query head, parity of j) per warp, lane = 4 dims: a warp reads
+// whole partial rows (coalesced), all of its up to 8 partials in flight at
+// once; the two parities combine through `scratch` (shared, 2 x 8 x
+// kPartialStride floats).  Partials come from other CTAs: loads bypass L1.
+__device__ __noinline__ void merge_partials(const float* head_parts, int first, int count,
+                                            float* dst, float (*o_rot)[kD], float* scratch) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int item = warp; item < 16; item += nwarps) {
+    const int hh = item >> 1, sub = item & 1;
+    float2 ml[kMergeGroup / 2];
     float4 oj[kMergeGroup / 2];
 #pragma unroll
-    for (int k = 0; k < kMergeGroup / 2; ++k) {
-      const int j = sub + 2 * k;
-      mj[k] = -1e30f;
-      lj[k] = 0.f;
-      oj[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b = 0; b < kMergeGroup / 2; ++b) {
+      const int j = sub + 2 * b;
+      ml[b] = make_float2(-1e30f, 0.f);
+      oj[b] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < count) {
         const float* pj = head_parts + ((size_t)(first + j) * 8 + hh) * kPartialStride;
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(pj));
-        mj[k] = ml.x;
-        lj[k] = ml.y;
-        oj[k] = __ldcg(reinterpret_cast<const float4*>(pj + 4) + d4);
+        ml[b] = __ldcg(reinterpret_cast<const float2*>(pj));
+        oj[b] = __ldcg(reinterpret_cast<const float4*>(pj + 4) + lane);
       }
     }
-    float M = mj[0];
+    float M = ml[0].x;
 #pragma unroll
-    for (int k = 1; k < kMergeGroup / 2; ++k) M = fmaxf(M, mj[k]);
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+    for (int b = 1; b < kMergeGroup / 2; ++b) M = fmaxf(M, ml[b].x);
     float L = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < kMergeGroup / 2; ++k) {
-      const float w = exp2f(mj[k] - M);
-      L = fmaf(w, lj[k], L);
-      o.x = fmaf(w, oj[k].x, o.x);
-      o.y = fmaf(w, oj[k].y, o.y);
-      o.z = fmaf(w, oj[k].z, o.z);
-      o.w = fmaf(w, oj[k].w, o.w);
+    for (int b = 0; b < kMergeGroup / 2; ++b) {
+      const float w = exp2f(ml[b].x - M);
+      L = fmaf(w, ml[b].y, L);
+      o.x = fmaf(w, oj[b].x, o.x);
+      o.y = fmaf(w, oj[b].y, o.y);
+      o.z = fmaf(w, oj[b].z, o.z);
+      o.w = fmaf(w, oj[b].w, o.w);
     }
-    L += __shfl_xor_sync(0xffffffffu, L, 1);
-    o.x += __shfl_xor_sync(0xffffffffu, o.x, 1);
-    o.y += __shfl_xor_sync(0xffffffffu, o.y, 1);
-    o.z += __shfl_xor_sync(0xffffffffu, o.z, 1);
-    o.w += __shfl_xor_sync(0xffffffffu, o.w, 1);
-    if (sub == 0) {
-      if (dst) {
-        float* pd = dst + hh * kPartialStride;
-        reinterpret_cast<float4*>(pd + 4)[d4] = o;
-        if (d4 == 0) {
-          pd[0] = M;
-          pd[1] = L;
-        }
-      } else {
-        const float inv = 1.f / L;
-        *reinterpret_cast<float4*>(&o_rot[hh][4 * d4]) =
-            make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
-      }
+    float* sc = scratch + (size_t)(sub * 8 + hh) * kPartialStride;
+    reinterpret_cast<float4*>(sc + 4)[lane] = o;
+    if (lane == 0) *reinterpret_cast<float2*>(sc) = make_float2(M, L);
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 8 * 32; idx += blockDim.x) {
+    const int hh = idx >> 5, d4 = idx & 31;
+    const float* s0 = scratch + (size_t)hh * kPartialStride;
+    const float* s1 = scratch + (size_t)(8 + hh) * kPartialStride;
+    const float2 ml0 = *reinterpret_cast<const float2*>(s0), ml1 = *reinterpret_cast<const float2*>(s1);
+    const float4 o0 = reinterpret_cast<const float4*>(s0 + 4)[d4];
+    const float4 o1 = reinterpret_cast<const float4*>(s1 + 4)[d4];
+    const float M = fmaxf(ml0.x, ml1.x), w0 = exp2f(ml0.x - M), w1 = exp2f(ml1.x - M);
+    const float L = w0 * ml0.y + w1 * ml1.y;
+    const float4 o = make_float4(w0 * o0.x + w1 * o1.x, w0 * o0.y + w1 * o1.y, w0 * o0.z + w1 * o1.z,
+                                 w0 * o0.w + w1 * o1.w);
+    if (dst) {
+      float* pd = dst + hh * kPartialStride;
+      reinterpret_cast<float4*>(pd + 4)[d4] = o;
+      if (d4 == 0) *reinterpret_cast<float2*>(pd) = make_float2(M, L);
+    } else {
+      const float inv = 1.f / L;
+      *reinterpret_cast<float4*>(&o_rot[hh][4 * d4]) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     }
   }
 }
@@ -505,6 +512,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
   __syncthreads();  // M_h^T and the partial sums are dead: stages >= 1 may load
   if (wh == 0 && lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   first_loads(1, stages);
+  if (tid < m.n_groups) {
+    const int gi = tid;
+    s.gdesc[gi] = make_uint2((2u * m.grp_width[gi] + (m.grp_split[gi] & 1u)) |
+                                 ((uint32_t)m.grp_kt0[gi] << 8) | ((uint32_t)m.grp_kt1[gi] << 16),
+                             (uint32_t)m.slot_koff[m.grp_first_slot[gi]]);
+  }
   // B fragments (query) of every decode k-tile; slots past the k-tile's run are zero
   for (int idx = tid; idx < m.n_ktiles * 32; idx += blockDim.x) {
     const int kt = idx >> 5, ln = idx & 31, gg = ln >> 2, tt = ln & 3;
@@ -543,18 +556,20 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
       for (int r = 0; r < 4; ++r) S[mt][r] = 0.f;
+#pragma unroll 1
     for (int gi = 0; gi < m.n_groups; ++gi) {
-      const int W = m.grp_width[gi], split = m.grp_split[gi];
-      const int kt0 = m.grp_kt0[gi], kt1 = m.grp_kt1[gi];
+      // group descriptor: 2 width + split | kt0 << 8 | kt1 << 16, first slot's byte offset
+      const uint2 desc = s.gdesc[gi];
+      const int W = (desc.x >> 1) & 0xf;
       // lane portion of slot t: 16W bits at byte 16W t + 2W g; this warp's half: + W wh
-      const int koff_lane = m.slot_koff[m.grp_first_slot[gi]] + W * (16 * t + 2 * g + wh);
-      switch (2 * W + split) {
-#define GTQ_GROUP(WW)                                                        \
-  case 2 * WW:                                                               \
-    group_scores<WW, false>(s, tl, kt0, kt1, koff_lane, lane4, lane, C);     \
-    break;                                                                   \
-  case 2 * WW + 1:                                                           \
-    group_scores<WW, true>(s, tl, kt0, kt1, koff_lane, lane4, lane, C);      \
+      const int koff_lane = (int)desc.y + W * (16 * t + 2 * g + wh);
+      switch (desc.x & 0x1f) {  // 2 W + split
+#define GTQ_GROUP(WW)                                                          \
+  case 2 * WW:                                                                 \
+    group_scores<WW, false>(s, tl, desc, koff_lane, lane4, lane, C);           \
+    break;                                                                     \
+  case 2 * WW + 1:                                                             \
+    group_scores<WW, true>(s, tl, desc, koff_lane, lane4, lane, C);            \
     break;
         GTQ_GROUP(1) GTQ_GROUP(2) GTQ_GROUP(3) GTQ_GROUP(4)
         GTQ_GROUP(5) GTQ_GROUP(6) GTQ_GROUP(7) GTQ_GROUP(8)
@@ -726,6 +741,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
   // second-level partial, and the last group to finish merges those.  Arrival
   // order comes from per-head tickets (acquire-release atomics); the last
   // arriver resets its ticket for the next call.
+  float* mscratch = wo;  // the warps' o are consumed: merge scratch
   bool finish = S == 1;
   if (!finish) {
     unsigned* tickets = a.tickets + (size_t)head * (1 + kMaxMergeGroups);
@@ -734,13 +750,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
     const int n1 = min(kMergeGroup, S - grp * kMergeGroup);
     if (arrive_last(&tickets[1 + grp], (unsigned)n1, &s.flag)) {
       if (n_groups == 1) {
-        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qs);
+        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qs, mscratch);
         finish = true;
       } else {
         merge_partials(head_parts, grp * kMergeGroup, n1,
-                       head_parts + (size_t)(kMaxSplits + grp) * 8 * kPartialStride, nullptr);
+                       head_parts + (size_t)(kMaxSplits + grp) * 8 * kPartialStride, nullptr,
+                       mscratch);
         if (arrive_last(&tickets[0], (unsigned)n_groups, &s.flag)) {
-          merge_partials(head_parts, kMaxSplits, n_groups, nullptr, s.qs);
+          merge_partials(head_parts, kMaxSplits, n_groups, nullptr, s.qs, mscratch);
           finish = true;
         }
       }
@@ -818,17 +835,16 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   const size_t stride = (p->tile_bytes + 127) & ~size_t(127);
   int dev_smem = 0;
   cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
-  // Stage area: the tile stages; at the end R_V and the warps' o; at setup,
-  // the setup scratch (M_h^T and the rotation's partial sums) at its top, clear
-  // of stage 0.  Three stages per pair when all pairs fit with them, else two,
-  // with as many pairs as fit.
+  // Stage area: the tile stages (two per pair, as many pairs as fit); at the
+  // end R_V, the warps' o and the merge scratch; at setup, the setup scratch
+  // (M_h^T and the rotation's partial sums) at its top, clear of stage 0.
   constexpr size_t kSetupScratch = (size_t)kD * kD * 4 + (size_t)4 * 8 * kD * 4;
   auto area_for = [&](int np_, int st_) {
     return std::max({stride * np_ * st_, (size_t)kD * kD * 4 + (size_t)2 * np_ * 8 * kD * 4,
                      stride * np_ + kSetupScratch});
   };
-  int stages = kMaxStages, np = kPairs;
-  if (stage_off + area_for(np, stages) > (size_t)dev_smem) stages = 2;
+  const int stages = kMaxStages;
+  int np = kPairs;
   while (np > 1 && stage_off + area_for(np, stages) > (size_t)dev_smem) --np;
   if (stage_off + area_for(np, stages) > (size_t)dev_smem) return cudaErrorInvalidValue;
   a.stages = stages;
