@@ -476,14 +476,6 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     const int norm_off = ROLE == 0 ? 1024 * (a.kb + a.vb) + 128 : 1024 * (a.kb + a.vb);
     const int jj = j & 63, npos = 2 * ((jj & 7) * 8 + (jj >> 3));
     const int n_chunks = gi.n_chunks;
-    uint32_t cgw[(kMaxChunks + 7) / 8];  // group of chunk c: 4 bits at (c % 8) * 4 of word c / 8
-#pragma unroll
-    for (int w = 0; w < (kMaxChunks + 7) / 8; ++w) {
-      cgw[w] = 0u;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (8 * w + k < n_chunks) cgw[w] |= (uint32_t)gi.chunk_group[8 * w + k] << (4 * k);
-    }
     int ovf = 0, it = 0;
     for (int64_t t = cta; t < n_mt; t += n_cta, ++it) {
       const int st = it % kStages, par = it & 1;
@@ -498,39 +490,58 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
           a.packed + ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + (j >> 6))) * a.tile_bytes;
       const uint8_t* xt = sm + kOffA + st * kStageBytes;
       float* sc_par = scale + par * kMaxGroups * kScaleStride;
-      // group sums of exact squares in fp32 (eight accumulators; a group's index is
-      // uniform, so its sum lands in a register through predicated moves)
-      float Sg[kMaxGroups];
-#pragma unroll
-      for (int g = 0; g < kMaxGroups; ++g) Sg[g] = 0.f;
+      // Group sums of exact squares in fp32 (eight accumulators), and each group's
+      // norm finished as soon as its sum is complete.  acc[i] held `terms` exact
+      // squares: |n / ||x|| - 1| <= (terms + 2) / 2 + 1/2 units of 2^-24 (sum depth
+      // terms - 1 + 3, halved by the root, plus its rounding); lo / hi add one each.
+      // A group whose fp16 rounding that window leaves open is settled below.
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      unsigned ambm = 0, zm = 0;  // 2 bits per group: 1 fp16 rounding undecided, 2 overflow undecided
+      uint32_t lh[kMaxGroups];    // fp16 candidates lo | hi << 16 of each group
       auto put = [&](int g) {
         const float S = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 #pragma unroll
-        for (int gg = 0; gg < kMaxGroups; ++gg)
-          if (gg == g) Sg[gg] = S;
-#pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        const int terms = ROLE == 0 ? gi.grp_chunks[g] : 16;
+        const float n = sqrtf(S);
+        float r;
+        asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(S));
+        const float delta = (0.5f * (float)terms + 4.f) * 5.9604645e-8f;
+        const float lo = n * (1.f - delta), hi = n * (1.f + delta);
+        const bool zero = S == 0.f, over = lo > 65504.f, strad = !over && hi > 65504.f;
+        const uint16_t l16 = __half_as_ushort(__float2half_rn(fminf(lo, 65504.f)));
+        const uint16_t h16 = __half_as_ushort(__float2half_rn(fminf(hi, 65504.f)));
+        zm |= zero ? 1u : 0u;
+        ovf |= over ? 1 : 0;
+        ambm |= ((zero || over) ? 0u : (strad ? 2u : (l16 != h16 ? 1u : 0u))) << (2 * g);
+        const uint32_t pk = (uint32_t)l16 | ((uint32_t)h16 << 16);
+#pragma unroll
+        for (int gg = 0; gg < kMaxGroups; ++gg)
+          if (gg == g) lh[gg] = pk;
+        *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) =
+            zero ? (uint16_t)0 : (over ? (uint16_t)0x7BFF : l16);
+        // scale of the codes (fp32, about 2^-22 relative)
+        sc_par[g * kScaleStride + j] = zero ? 0.f : gi.sqrt_m[g] * r;
       };
       int ng;
       if (ROLE == 0) {
         // gathered exact inputs, 8 columns per chunk, 8 chunks per wait
         ng = gi.n_groups;
         int cur = 0;
-#pragma unroll
-        for (int w = 0; w < (kMaxChunks + 7) / 8; ++w) {
-          const int b = 8 * w;
-          if (b >= n_chunks) break;
+        // a loop, not unrolled: this warp's code must stay small next to the code warps'
+#pragma unroll 1
+        for (int b = 0; b < n_chunks; b += 8) {
           uint32_t r0[32], r1[32];
           tc_ld32(trow + 8 * b, r0);
           tc_ld32(trow + 8 * b + 32, r1);
           tc_wait_ld();
+          const uint2 cg = *reinterpret_cast<const uint2*>(&gi.chunk_group[b]);  // groups of chunks b..b+7
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             if (b + k < n_chunks) {
-              const int g = (int)((cgw[w] >> (4 * k)) & 15u);
+              const int g = (int)(((k < 4 ? cg.x : cg.y) >> (8 * (k & 3))) & 0xffu);
               if (g != cur) {
                 put(cur);
                 cur = g;
@@ -563,42 +574,17 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
         }
         put(0);
       }
-      // every group's norm at once (independent chains).  acc[i] held `terms` exact
-      // squares: |n / ||x|| - 1| <= (terms + 2) / 2 + 1/2 units of 2^-24 (sum depth
-      // terms - 1 + 3, halved by the root, plus its rounding); lo / hi add one each
-      uint16_t hb[kMaxGroups], hl[kMaxGroups], hh[kMaxGroups];
-      float sv[kMaxGroups];
-      unsigned ambm = 0, zm = 0;  // 2 bits per group: 1 fp16 rounding undecided, 2 overflow undecided
-#pragma unroll
-      for (int g = 0; g < kMaxGroups; ++g) {  // all eight computed (unused groups have S = 0)
-        const float S = Sg[g];
-        const int terms = ROLE == 0 ? gi.grp_chunks[g] : 16;
-        const float n = sqrtf(S);
-        float r;
-        asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(S));
-        const float delta = (0.5f * (float)terms + 4.f) * 5.9604645e-8f;
-        const float lo = n * (1.f - delta), hi = n * (1.f + delta);
-        const bool live = g < ng;
-        const bool zero = S == 0.f, over = lo > 65504.f, strad = !over && hi > 65504.f;
-        const uint16_t l16 = __half_as_ushort(__float2half_rn(fminf(lo, 65504.f)));
-        const uint16_t h16 = __half_as_ushort(__float2half_rn(fminf(hi, 65504.f)));
-        hl[g] = l16;
-        hh[g] = h16;
-        hb[g] = zero ? (uint16_t)0 : (over ? (uint16_t)0x7BFF : l16);
-        sv[g] = zero ? 0.f : gi.sqrt_m[g] * r;  // scale of the codes (fp32, about 2^-22 relative)
-        if (live) {
-          zm |= zero ? 1u : 0u;
-          ovf |= over ? 1 : 0;
-          ambm |= (zero || over) ? 0u : (strad ? 2u : (l16 != h16 ? 1u : 0u)) << (2 * g);
-        }
-      }
       const unsigned zero_any = __ballot_sync(0xffffffffu, zm != 0);
       if (__ballot_sync(0xffffffffu, ambm != 0)) {
-#pragma unroll
-        for (int g = 0; g < kMaxGroups; ++g) {
-          if (g >= ng) break;
+#pragma unroll 1
+        for (int g = 0; g < ng; ++g) {
           const unsigned amb_g = (ambm >> (2 * g)) & 3u;
           unsigned am = __ballot_sync(0xffffffffu, amb_g != 0);
+          uint32_t pk = lh[0];
+#pragma unroll
+          for (int gg = 1; gg < kMaxGroups; ++gg)
+            if (gg == g) pk = lh[gg];
+          const uint16_t hlg = (uint16_t)(pk & 0xffffu), hhg = (uint16_t)(pk >> 16);
           while (am) {  // exact decision from the fp64 sum of squares, the whole warp helping
             const int src = __ffs(am) - 1;
             am &= am - 1;
@@ -614,28 +600,24 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
 #pragma unroll
             for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
             if (lane == src) {
-              if (amb_g == 1 && hh[g] == hl[g] + 1) {
+              uint16_t hb;
+              if (amb_g == 1 && hhg == hlg + 1) {
                 // n is between the two fp16 values: compare with their midpoint squared
                 // (12 significant bits, exact in fp64); a tie rounds to even
-                const double mid = 0.5 * ((double)__half2float(__ushort_as_half(hl[g])) +
-                                          (double)__half2float(__ushort_as_half(hh[g])));
+                const double mid = 0.5 * ((double)__half2float(__ushort_as_half(hlg)) +
+                                          (double)__half2float(__ushort_as_half(hhg)));
                 const double m2 = mid * mid;
-                hb[g] = sq > m2 ? hh[g] : (sq < m2 ? hl[g] : ((hl[g] & 1) ? hh[g] : hl[g]));
+                hb = sq > m2 ? hhg : (sq < m2 ? hlg : ((hlg & 1) ? hhg : hlg));
               } else {
                 const double n64 = sqrt(sq);
                 if (n64 > 65504.0) ovf = 1;
-                hb[g] = __half_as_ushort(__double2half(n64 > 65504.0 ? 65504.0 : n64));
+                hb = __half_as_ushort(__double2half(n64 > 65504.0 ? 65504.0 : n64));
               }
+              *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb;
             }
           }
         }
       }
-#pragma unroll
-      for (int g = 0; g < kMaxGroups; ++g)
-        if (g < ng) {
-          *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb[g];
-          sc_par[g * kScaleStride + j] = sv[g];
-        }
       if (lane == 0) zflags[par * 4 + q] = zero_any ? 1 : 0;
       tc_fence_before();
       __syncwarp();
