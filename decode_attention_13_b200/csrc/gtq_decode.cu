@@ -28,7 +28,8 @@ namespace {
 constexpr int kPairs = 8;  // one CTA per SM: up to 8 warp pairs, 2 tile stages per pair
 constexpr int kWarps = 2 * kPairs;
 constexpr int kMaxStages = 2;  // tile stages per warp pair
-constexpr unsigned kSpinLimit = 1u << 26;
+constexpr uint32_t kSuspendHintNs = 1000000;  // mbarrier try_wait suspend-time hint
+constexpr uint64_t kWaitNs = 2000000000ull;    // bound of one wait
 
 struct DecodeArgs {
   const uint8_t* packed;
@@ -90,19 +91,29 @@ __device__ inline void tile_load(void* dst, const void* src, unsigned bytes, uin
       : "memory");
 }
 
-// bounded wait on an mbarrier phase; returns false if the bound expired
+// bounded wait on an mbarrier phase; returns false after about two seconds.
+// Each try suspends the thread until the phase completes or a time hint
+// expires, so a waiting warp takes no issue slots from the working ones.
 __device__ inline bool mbar_wait(uint64_t* bar, unsigned phase) {
-  for (unsigned i = 0; i < kSpinLimit; ++i) {
+  uint64_t t0 = 0;
+  for (unsigned i = 0;; ++i) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(kSuspendHintNs)
         : "memory");
     if (ok) return true;
+    if ((i & 15u) == 15u) {
+      uint64_t now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t0 == 0)
+        t0 = now;
+      else if (now - t0 > kWaitNs)
+        return false;
+    }
   }
-  return false;
 }
 
 __device__ inline void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {

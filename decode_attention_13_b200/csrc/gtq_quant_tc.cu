@@ -45,6 +45,7 @@ constexpr int kTcWarps = 14;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kMTile = 128;          // tokens per MMA tile (= 2 packed tiles)
 constexpr int kStages = 3;           // input tile stages
+constexpr uint32_t kSuspendHintNs = 1000000;  // mbarrier try_wait suspend-time hint
 constexpr int kKeyShare = 67;        // percent of a head's CTAs that quantize keys
 constexpr uint64_t kTcWaitNs = 2000000000ull;  // bound of every barrier wait
 
@@ -127,19 +128,21 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-// bounded wait: gives up (returns false) after about two seconds
+// bounded wait: gives up (returns false) after about two seconds.  Each try
+// suspends the thread until the phase completes or a time hint expires, so a
+// waiting warp takes no issue slots from the working ones.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   uint64_t t0 = 0;
   for (unsigned i = 0;; ++i) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     if (ok) return true;
-    if ((i & 255u) == 255u) {
+    if ((i & 15u) == 15u) {
       uint64_t now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0)
