@@ -161,7 +161,8 @@ GTQ_API int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_d
  *   T           1 <= T <= t_capacity.
  *   q_dev       post-RoPE queries [batch][n_q_heads][128], q_dtype, contiguous,
  *               16-byte aligned.  Query head hq uses KV head hq / (Hq / Hkv).
- *   out_dev     fp32 [batch][n_q_heads][128], contiguous, written in full.
+ *   out_dev     fp32 [batch][n_q_heads][128], contiguous, 16-byte aligned, written
+ *               in full.
  * Uses the plan's workspace: concurrent decodes on one plan must not overlap.
  * Errors: INVALID, UNSUPPORTED (head_dim != 128), STATE, CUDA.
  */
