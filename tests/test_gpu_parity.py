@@ -149,6 +149,9 @@ def check_case(case, check_decode=True, quantized=False):
     (1, 1, 8, 200, 1, 1, 0, "fp16"),
     (1, 1, 8, 190, 8, 8, 1, "fp16"),
     (1, 1, 5, 257, 5, 3, 0, "fp32"),
+    # wide tiles: fewer warp pairs per CTA, with enough tiles for two merge levels
+    (1, 1, 8, 8192, 8, 8, 0, "fp16"),
+    (2, 1, 4, 4000, 8, 6, 1, "fp16"),
 ])
 def test_layer_parity(B, hkv, gq, T, kb, vb, pairing, dtype):
     check_case(Case(B, hkv, gq, T, kb, vb, pairing, dtype, seed=100 + T))
