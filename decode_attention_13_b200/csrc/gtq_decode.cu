@@ -50,6 +50,7 @@ struct DecodeArgs {
   int kb, vb;
   int splits;
   int stages;         // tile stages per warp pair
+  int area;           // bytes of the stage area
   int rot_off;        // byte offset of the setup scratch in the stage area
   int64_t tiles_T;    // ceil(T / 64)
 };
@@ -151,7 +152,6 @@ __device__ inline uint32_t pack_half2(__half lo, __half hi) {
 static_assert(sizeof(HeadMeta) % 16 == 0, "metadata is bulk-copied");
 
 struct DecodeSmem {
-  uint32_t tab[kDecodeImageBytes / 4];
   uint4 qf[kMaxKt][32];  // per k-tile & lane: hi(slot A), hi(slot B), lo(A), lo(B)
   alignas(16) HeadMeta meta;
   uint2 gdesc[kMaxGroups];  // per key group: 2 width + split | kt0 << 8 | kt1 << 16; byte offset
@@ -184,25 +184,30 @@ __device__ __forceinline__ uint32_t fld(const uint32_t* x, uint32_t orv) {
   return (v & mask) | orv;
 }
 
+// Table load from a shared-window address: `addr` already holds the table
+// base (8 KB aligned) ORed with the lane and the index; the region offset is
+// the load's immediate.
 template <uint32_t OFF>
-__device__ __forceinline__ uint32_t lds_tab(const DecodeSmem& s, uint32_t idx) {
-  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(s.tab) + OFF + idx);
+__device__ __forceinline__ uint32_t lds_tab(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+  return v;
 }
 
 // hi|lo word (fp16 hi in the low half) of the code of width W at bits [P, P + W)
 template <int W, int P>
 __device__ __forceinline__ uint32_t single_code(const DecodeSmem& s, const uint32_t* x, uint32_t lane4) {
   if constexpr (W >= 4 && W <= 6)
-    return lds_tab<kLaneSingleOff(W)>(s, fld<P, W, 7>(x, lane4));
+    return lds_tab<kLaneSingleOff(W)>(fld<P, W, 7>(x, lane4));
   else
-    return lds_tab<kSharedSingles + kSingleOff(W)>(s, fld<P, W, 2>(x, 0u));
+    return lds_tab<kSharedSingles + kSingleOff(W)>(fld<P, W, 2>(x, lane4 & ~127u));
 }
 
 // half2 (hi parts) of codes (2X, 2X + 1), width W, from the bit string x
 template <int W, int X>
 __device__ __forceinline__ uint32_t pair_hi(const DecodeSmem& s, const uint32_t* x, uint32_t lane4) {
   if constexpr (W <= 3) {
-    return lds_tab<kPairOff(W)>(s, fld<2 * X * W, 2 * W, 7>(x, lane4));
+    return lds_tab<kPairOff(W)>(fld<2 * X * W, 2 * W, 7>(x, lane4));
   } else {
     const uint32_t e0 = single_code<W, 2 * X * W>(s, x, lane4);
     const uint32_t e1 = single_code<W, (2 * X + 1) * W>(s, x, lane4);
@@ -430,6 +435,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
   float* rot_part = mt + kD * kD;                                 // [4][8][128]
   float(*qt)[8] = reinterpret_cast<float(*)[8]>(&s.qs[0][0]);    // q^T [dim][head]
 
+  // lookup tables after the stage area, at an 8 KB-aligned shared address (so
+  // that table base, index and lane combine by OR)
+  const uint32_t raw_sa = smem_u32(smem_raw);
+  const uint32_t tab_sa = (raw_sa + (uint32_t)(stage_off + a.area) + 8191u) & ~8191u;
+  uint8_t* tab = smem_raw + (tab_sa - raw_sa);
+
   // Setup: lookup tables, head metadata and M_h^T by bulk copies (issued
   // first: nothing here depends on the previous grid), then stage 0 of every
   // pair; the queries follow the grid-dependency wait.
@@ -444,7 +455,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&s.setup_bar)),
                  "r"((unsigned)(kDecodeImageBytes + sizeof(HeadMeta) + kD * kD * sizeof(float)))
                  : "memory");
-    bulk_copy(s.tab, a.dec_image, kDecodeImageBytes, &s.setup_bar);
+    bulk_copy(tab, a.dec_image, kDecodeImageBytes, &s.setup_bar);
     bulk_copy(&s.meta, a.meta + head, sizeof(HeadMeta), &s.setup_bar);
     bulk_copy(mt, a.mrow_t + (size_t)head * kD * kD, kD * kD * sizeof(float), &s.setup_bar);
   }
@@ -454,7 +465,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_kernel(DecodeArgs a) {
   const HeadMeta& m = s.meta;
   const int load_bytes = 1024 * (a.kb + VB) + 128 + 128 * m.n_groups;
   const int knorm_off = 1024 * (a.kb + VB) + 128, vnorm_off = 1024 * (a.kb + VB);
-  const uint32_t lane4 = (uint32_t)lane << 2;
+  // lookup-table base | lane * 4: the high bits of every table address
+  const uint32_t lane4 = tab_sa | ((uint32_t)lane << 2);
 
   // tiles of this split, dealt to warp pairs round-robin
   const int64_t per = (a.tiles_T + a.splits - 1) / a.splits;
@@ -854,15 +866,17 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
     return std::max({stride * np_ * st_, (size_t)kD * kD * 4 + (size_t)2 * np_ * 8 * kD * 4,
                      stride * np_ + kSetupScratch});
   };
+  constexpr size_t kTables = (size_t)kDecodeImageBytes + 8192;  // + alignment slack
   const int stages = kMaxStages;
   int np = kPairs;
-  while (np > 1 && stage_off + area_for(np, stages) > (size_t)dev_smem) --np;
-  if (stage_off + area_for(np, stages) > (size_t)dev_smem) return cudaErrorInvalidValue;
+  while (np > 1 && stage_off + area_for(np, stages) + kTables > (size_t)dev_smem) --np;
+  if (stage_off + area_for(np, stages) + kTables > (size_t)dev_smem) return cudaErrorInvalidValue;
   a.stages = stages;
   const int nw = 2 * np;
   const size_t area = area_for(np, stages);
   a.rot_off = (int)(area - kSetupScratch);
-  const size_t smem = stage_off + area;
+  a.area = (int)area;
+  const size_t smem = stage_off + area + kTables;
   int per_sm = 1;
   switch (a.vb) {
 #define GTQ_OCC_VB(VB)                                                                           \
