@@ -52,7 +52,6 @@ void release(gtq_plan* p) {
   cudaFree(p->d_mrow);
   cudaFree(p->d_mrow_t);
   cudaFree(p->d_bimg);
-  cudaFree(p->d_qrot);
   cudaFree(p->d_partials);
   cudaFree(p->d_tickets);
   cudaFree(p->d_status);
@@ -92,7 +91,6 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
   alloc((void**)&p->d_mrow_t, H * kD * kD * sizeof(float));
   if (cfg->head_dim == kD) alloc((void**)&p->d_bimg, H * b_image_bytes());
-  alloc((void**)&p->d_qrot, H * 8 * kD * sizeof(float));
   alloc((void**)&p->d_partials, H * kPartialSlots * 8 * kPartialStride * sizeof(float));
   alloc((void**)&p->d_tickets, H * (1 + kMaxMergeGroups) * sizeof(unsigned));
   alloc((void**)&p->d_status, sizeof(int));

@@ -109,8 +109,6 @@ struct Tables {
   float* rot_v;      // R_V 128 x 128 row-major (fp32)
   double* dist;      // D(0..8)
   float* thr;        // fp32 thresholds, width w at thr_base(w)
-  __half* lut_hi;    // fp16(centroid), width w at lut_base(w)
-  __half* lut_lo;    // fp16(centroid - fp16(centroid))
   uint4* dec_image;  // kDecodeImageBytes: the decode kernel's lookup tables
   uint8_t* rv_image; // R_V as the quantizer's tensor-core B operand (fp16 hi + lo, 64 KB)
   uint8_t* code_lut; // kCodeLutBytes: CodeLutMeta + cells (built on the device from thr)
@@ -143,7 +141,6 @@ struct gtq_plan {
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
   float* d_mrow_t;    // [heads][128][128] the same, transposed: [dim][packed position]
   uint8_t* d_bimg;    // [heads] M_h as the quantizer's tensor-core B operand (64 KB each)
-  float* d_qrot;      // [heads][8][128] rotated, scaled queries (decode workspace)
   float* d_partials;  // [heads][kPartialSlots][8][kPartialStride]
   unsigned* d_tickets;  // [heads][1 + kMaxMergeGroups] arrival counters of the split merge
   int* d_status;      // device status word

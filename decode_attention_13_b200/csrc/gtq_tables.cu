@@ -279,8 +279,6 @@ int tables_for(int device, uint64_t seed, Tables* out) {
   if (e == cudaSuccess) e = up((void**)&t.rot_v, rv.data(), rv.size() * sizeof(float));
   if (e == cudaSuccess) e = up((void**)&t.dist, dist.data(), dist.size() * sizeof(double));
   if (e == cudaSuccess) e = up((void**)&t.thr, thr.data(), thr.size() * sizeof(float));
-  if (e == cudaSuccess) e = up((void**)&t.lut_hi, lhi.data(), lhi.size() * sizeof(__half));
-  if (e == cudaSuccess) e = up((void**)&t.lut_lo, llo.data(), llo.size() * sizeof(__half));
   if (e == cudaSuccess) e = up((void**)&t.dec_image, img.data(), img.size() * sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMalloc((void**)&t.rv_image, b_image_bytes());
   if (e == cudaSuccess) e = build_b_images(t.rot_v, 1, 0, t.rv_image, 0);
