@@ -1,21 +1,22 @@
 // Fused GQA decode attention over the Block-GTQ packed cache ("RoPE-Aware Bit
 // Allocation for KV-Cache Quantization", Abstract: the "packed-cache serving
 // path").  No fp16 K or V is materialised: codes are turned into tensor-core
-// operands in registers.
-//
-//   rotate_q_kernel  q_rot[pos] = M_h[pos] . q * log2(e) / (sqrt(d) sqrt(m_g)):
-//                    every query head of a KV head rotated once per call.
-//   decode_kernel    split-K over the context.  A warp owns 64-token tiles
-//                    staged by 1-D bulk TMA (cp.async.bulk + mbarrier).  Scores:
-//                    mma.m16n8k16 with A = codebook values of 16 tokens x 16
-//                    rotated coords and B = q_rot (8 query heads), accumulated
-//                    per group and scaled by the fp16 group norms; the widest
-//                    groups use split fp16 (hi/lo) operands.  Online softmax in
-//                    base 2.  P.V: mma with A = V codebook values (16 dims x 16
-//                    tokens) and B = P^T (movmatrix transpose of the score
-//                    fragment), accumulated in V's rotated basis.
-//   merge_kernel     merge of the split partials (m, l, o) per query head and
-//                    o = R_V^T o_rot / l.
+// operands in registers.  One launch per call (decode_kernel), grid = (context
+// splits, heads), one CTA per SM:
+//   setup   lookup tables, head metadata and M_h^T by bulk copies; after the
+//           grid-dependency wait the query heads of the KV head are rotated
+//           once, q_rot[pos] = M_h[pos] . q * log2(e) / (sqrt(d) sqrt(m_g)).
+//   loop    the split's 64-token tiles, each shared by a pair of warps (32
+//           tokens each) and staged by 1-D bulk TMA (cp.async.bulk + mbarrier).
+//           Scores: mma.m16n8k16 with A = codebook values of 16 tokens x 16
+//           rotated coords and B = q_rot (8 query heads), accumulated per key
+//           group and scaled by its fp16 norms; the widest groups use split
+//           fp16 (hi/lo) operands.  Online softmax in base 2.  P.V: mma with
+//           A = V codebook values (16 dims x 16 tokens) and B = P^T (movmatrix
+//           transpose of the score fragment), accumulated in V's rotated basis.
+//   merge   the CTA's warps, then the splits: the last CTA of each group of
+//           splits merges the group, the last group merges the rest and writes
+//           o = R_V^T o_rot / l.
 #include <algorithm>
 #include <cmath>
 #include <cstddef>

@@ -7,9 +7,9 @@
 // thresholds below (sqrt(m)/n) (M_h k)_j, fp16(n) stored; values likewise with
 // one group of 128 and R_V.
 //
-// One launch; a CTA works on one head in one role (keys or values; a head's CTAs
-// are shared between the roles by their cost per tile)
-// and walks 128-token tiles that lie inside the tokens being written.  Per tile:
+// One launch; a CTA works on one head in one role, keys or values (about two
+// thirds of a head's CTAs take keys, whose tiles cost more), and walks the
+// 128-token tiles that lie inside the tokens being written.  Per tile:
 //   * code GEMM   D_c[coord][token] = R . X^T with R = M_h (keys) or R_V (values)
 //                 split into fp16 hi + lo parts (A operand, resident in shared
 //                 memory) and X the fp16 tile (B operand, TMA, 128B swizzle);
@@ -17,8 +17,9 @@
 //   * gather GEMM D_p[token][row] = X . P^T with P a 0/1 matrix that lists the
 //                 dims of key group 0, then group 1, ... (each group padded to 8
 //                 rows); every output is one input element, so D_p holds the
-//                 exact fp16 inputs as fp32, grouped by key group.  For values P
-//                 is the identity.
+//                 exact fp16 inputs as fp32, grouped by key group.  Keys only:
+//                 the value norms are summed straight from the fp16 tile in
+//                 shared memory.
 // Warps: 0 TMA producer; 1 tensor-memory owner and MMA issuer; 2-5 norm warps
 // (thread = token: group sums of squares from D_p); 6-13 code warps (thread =
 // rotated coordinate, 64 tokens: codes, bit packing in registers with one
@@ -30,7 +31,8 @@
 // fp64 sum of squares of the fp16 tile in shared memory.  Scales for the codes
 // come from the same sum (approximate reciprocal root).  A tile that holds a zero
 // vector or group is flagged, and its codes are masked to 0.
-// Waits are bounded; on expiry the status word gets GTQ_ERR_TIMEOUT's bit.
+// Waits suspend the thread (mbarrier try_wait with a time hint) and are bounded;
+// on expiry the status word gets GTQ_ERR_TIMEOUT's bit.
 #include <cuda.h>
 
 #include <cmath>
