@@ -687,25 +687,21 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
 #pragma unroll
       for (int i = 0; i < 16; ++i) A[i] = 0;
       {
-        uint32_t y[32];
-        tc_ld32(tcol + (uint32_t)(ac * kD), y);
-        tc_wait_ld();
-        if (zmask)
-          code_half<ROLE, 0, true>(y, sc, L, A);
-        else
-          code_half<ROLE, 0, false>(y, sc, L, A);
-      }
-      {
-        uint32_t y[32];
-        tc_ld32(tcol + (uint32_t)(ac * kD) + 32, y);
+        // both halves of the accumulator in one wait, then release it at once
+        uint32_t y0[32], y1[32];
+        tc_ld32(tcol + (uint32_t)(ac * kD), y0);
+        tc_ld32(tcol + (uint32_t)(ac * kD) + 32, y1);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kCEmpty + ac));  // accumulator may be overwritten
-        if (zmask)
-          code_half<ROLE, 1, true>(y, sc + 32, L, A);
-        else
-          code_half<ROLE, 1, false>(y, sc + 32, L, A);
+        if (zmask) {
+          code_half<ROLE, 0, true>(y0, sc, L, A);
+          code_half<ROLE, 1, true>(y1, sc + 32, L, A);
+        } else {
+          code_half<ROLE, 0, false>(y0, sc, L, A);
+          code_half<ROLE, 1, false>(y1, sc + 32, L, A);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kSEmpty + par));  // scales and flags read
