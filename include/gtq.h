@@ -188,7 +188,9 @@ GTQ_API int gtq_get_bits(gtq_plan* plan, uint8_t* host_bits, void* stream);
 GTQ_API int gtq_get_energy(gtq_plan* plan, double* host_energy, void* stream);
 
 /* Read and clear the plan's device status word (synchronises the device):
- * GTQ_OK, GTQ_ERR_OVERFLOW or GTQ_ERR_TIMEOUT. */
+ * GTQ_OK, GTQ_ERR_OVERFLOW or GTQ_ERR_TIMEOUT.  After GTQ_ERR_TIMEOUT the
+ * outputs of the calls since the last check are undefined and so is the
+ * plan's split-merge state: free the plan and build a new one. */
 GTQ_API int gtq_status(gtq_plan* plan);
 
 /* Human-readable name of a return code (static string). */
