@@ -1,7 +1,7 @@
 // Block-GTQ allocation on the device ("RoPE-Aware Bit Allocation for KV-Cache
-// Quantization", Abstract: "a label-free energy score for each RoPE block",
-// "greedily allocates integer bit widths by marginal gain", per layer and KV
-// head).
+// Quantization", Abstract): per layer and KV head, an energy score of every
+// RoPE block that needs no labels, then integer widths given one bit at a time
+// to the block with the largest marginal gain.
 //
 //   energy_partial_kernel  E partial sums over token chunks, fp64, fixed order
 //   energy_finish_kernel   E_i = (sum over p0 and p1 of block i) / T
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
                                                    const double* __restrict__ rot_k, int pairing,
                                                    HeadMeta* __restrict__ meta_out,
                                                    float* __restrict__ mrow,
-                                                   float* __restrict__ mrow_t) {
+                                                   float* __restrict__ rotpack) {
   const int head = blockIdx.x;
   __shared__ HeadMeta m;
   __shared__ uint8_t grp_blocks[kMaxGroups][kBlocks];
@@ -212,12 +212,15 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
     m.reserved = 0;
   }
   __syncthreads();
-  // key rotation rows: M_h[pos][dim], pos = 2 * slot + e  <->  row r = 2 (slot - first) + e of R_m
+  // key rotation rows: M_h[pos][dim], pos = 2 * slot + e  <->  row r = 2 (slot - first) + e of R_m;
+  // the rotation pack: coord_dim[pos] and every group's R_m transposed
   const int pos = threadIdx.x;
   float* row = mrow + ((size_t)head * kD + pos) * kD;
-  float* col = mrow_t + (size_t)head * kD * kD + pos;  // M_h^T[dim][pos]
+  float* pack = rotpack + (size_t)head * kRotPackMaxWords;
+  uint8_t* coord_dim = reinterpret_cast<uint8_t*>(pack);
   for (int dd = 0; dd < kD; ++dd) row[dd] = 0.f;
   const int slot = pos >> 1;
+  uint8_t cdim = 0;
   if (slot < m.n_slots) {
     const int g = m.slot_group[slot];
     const int mm = m.grp_m[g];
@@ -225,13 +228,19 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
     size_t off = 0;
     for (int q = 2; q < mm; q += 2) off += (size_t)q * q;
     const double* R = rot_k + off + (size_t)r * mm;
+    size_t poff = kRotPackHeaderWords;  // this group's block in the pack
+    for (int gg = 0; gg < g; ++gg) poff += (size_t)m.grp_m[gg] * m.grp_m[gg];
     for (int c = 0; c < mm; ++c) {
       const int blk = grp_blocks[g][c >> 1], el = c & 1;
       const int dim = pairing == GTQ_PAIRING_HALF ? blk + el * kBlocks : 2 * blk + el;
       row[dim] = (float)R[c];
+      pack[poff + (size_t)c * mm + r] = (float)R[c];
     }
+    // coordinate r of the group (the same index range as its rows) has this dim
+    const int blk = grp_blocks[g][r >> 1], el = r & 1;
+    cdim = (uint8_t)(pairing == GTQ_PAIRING_HALF ? blk + el * kBlocks : 2 * blk + el);
   }
-  for (int dd = 0; dd < kD; ++dd) col[(size_t)dd * kD] = row[dd];
+  coord_dim[pos] = cdim;
   if (threadIdx.x == 0) meta_out[head] = m;
 }
 
@@ -265,7 +274,7 @@ cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s) {
       p->d_bits);
   if (p->cfg.head_dim == kD) {
     meta_kernel<<<p->n_heads, 128, 0, s>>>(p->d_bits, p->d_energy, p->tab.rot_k,
-                                           p->cfg.rope_pairing, p->d_meta, p->d_mrow, p->d_mrow_t);
+                                           p->cfg.rope_pairing, p->d_meta, p->d_mrow, p->d_rotpack);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return build_b_images(p->d_mrow, p->n_heads, (size_t)kD * kD, p->d_bimg, s);
@@ -332,14 +341,22 @@ extern "C" int gtq_block_energy_noalloc(const gtq_config* cfg, const void* k_dev
     return GTQ_ERR_INVALID;
   for (int i = 0; i < 3; ++i)
     if (k_strides[i] < 0 || (k_strides[i] * esz) % 16) return GTQ_ERR_INVALID;
-  const int heads = cfg->batch * cfg->n_kv_heads;
+  // heads is grid.y of both kernels: the product is formed in 64 bits and
+  // bounded by the grid limit before anything else uses it
+  const int64_t heads64 = (int64_t)cfg->batch * (int64_t)cfg->n_kv_heads;
+  if (heads64 > 65535) {
+    set_last_error("gtq_block_energy_noalloc: batch * n_kv_heads exceeds 65535");
+    return GTQ_ERR_INVALID;
+  }
+  const int heads = (int)heads64;
   const int64_t chunks = (T + kEnergyChunk - 1) / kEnergyChunk;
-  if ((double)heads * (double)chunks * 128.0 > (double)kNoAllocEnergyDoubles) {
+  if (chunks > (int64_t)kNoAllocEnergyDoubles ||
+      heads64 * chunks * 128 > (int64_t)kNoAllocEnergyDoubles) {
     char msg[160];
     snprintf(msg, sizeof(msg),
              "gtq_block_energy_noalloc: %d heads x %lld token chunks need %lld partial sums, "
              "the fixed scratch holds %zu",
-             heads, (long long)chunks, (long long)heads * chunks * 128, kNoAllocEnergyDoubles);
+             heads, (long long)chunks, (long long)(heads64 * chunks * 128), kNoAllocEnergyDoubles);
     set_last_error(msg);
     return GTQ_ERR_UNSUPPORTED;
   }

@@ -50,7 +50,7 @@ void release(gtq_plan* p) {
   cudaFree(p->d_bits);
   cudaFree(p->d_meta);
   cudaFree(p->d_mrow);
-  cudaFree(p->d_mrow_t);
+  cudaFree(p->d_rotpack);
   cudaFree(p->d_bimg);
   cudaFree(p->d_partials);
   cudaFree(p->d_tickets);
@@ -89,12 +89,12 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   alloc((void**)&p->d_bits, H * p->n_blocks);
   alloc((void**)&p->d_meta, H * sizeof(HeadMeta));
   alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
-  alloc((void**)&p->d_mrow_t, H * kD * kD * sizeof(float));
+  alloc((void**)&p->d_rotpack, H * kRotPackBytes);
   if (cfg->head_dim == kD) alloc((void**)&p->d_bimg, H * b_image_bytes());
   alloc((void**)&p->d_partials, H * kPartialSlots * 8 * kPartialStride * sizeof(float));
-  alloc((void**)&p->d_tickets, H * (1 + kMaxMergeGroups) * sizeof(unsigned));
+  alloc((void**)&p->d_tickets, H * kTicketStride * sizeof(unsigned));
   alloc((void**)&p->d_status, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * (1 + kMaxMergeGroups) * sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * kTicketStride * sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(p->d_meta, 0, H * sizeof(HeadMeta));
   if (e != cudaSuccess) {
@@ -231,6 +231,10 @@ int gtq_status(gtq_plan* plan) {
   if (e == cudaSuccess) e = cudaMemcpy(&v, plan->d_status, sizeof(int), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemset(plan->d_status, 0, sizeof(int));
   if (e != cudaSuccess) return GTQ_ERR_CUDA;
+  if (v & kStatusLayout) {
+    set_last_error("decode kernel: shared-memory window above the planned layout");
+    return GTQ_ERR_CUDA;
+  }
   if (v & kStatusTimeout) return GTQ_ERR_TIMEOUT;
   if (v & kStatusOverflow) return GTQ_ERR_OVERFLOW;
   return GTQ_OK;

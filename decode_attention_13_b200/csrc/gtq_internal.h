@@ -24,6 +24,7 @@ constexpr int kMaxMergeGroups = kMaxSplits / kMergeGroup;
 constexpr int kPartialSlots = kMaxSplits + kMaxMergeGroups;  // per head: level 1 + level 2
 constexpr int kStatusOverflow = 1;      // status word bits
 constexpr int kStatusTimeout = 2;
+constexpr int kStatusLayout = 4;        // a kernel found its shared-memory layout unusable
 
 // First LUT / threshold entry of width w (1..8).
 __host__ __device__ inline int lut_base(int w) { return (1 << w) - 2; }
@@ -53,35 +54,59 @@ struct HeadMeta {
   uint8_t kt_flags[kMaxKt];       // bit 0: first k-tile of its group, bit 1: last
 };
 
-// Decode lookup tables, laid out exactly as the decode kernel's shared memory.
-// Every table is addressed as "region offset + index", where the index is built
-// by one shift and one mask-or from the packed bits:
-//  * pair tables, widths 1..3: entry c0 | c1 << w holds the fp16 half2
-//    (cb[c0], cb[c1]) (hi parts); one copy per lane, at byte
-//    kPairOff(w) + entry * 128 + lane * 4, so a warp-wide lookup never has a
-//    bank conflict;
-//  * lane-private single-code tables, widths 4..6: entry c holds fp16 hi part
-//    (low half) and lo part (high half) of cb[c], at byte
-//    kLaneSingleOff(w) + c * 128 + lane * 4;
-//  * shared single-code tables, widths 1..8 (same entry format), at byte
-//    kSharedSingles + kSingleOff(w) + c * 4 (one copy; used for the lo parts of
-//    narrow split groups and for widths 7 and 8).
-constexpr int kDecodeImageBytes = 28672;
-__host__ __device__ constexpr uint32_t kPairOff(int w) { return w == 3 ? 0u : (w == 2 ? 8192u : 10240u); }
-__host__ __device__ constexpr uint32_t kLaneSingleOff(int w) {
-  return w == 4 ? 12288u : (w == 5 ? 24576u : 16384u);
+// Decode lookup tables, laid out exactly as the decode kernel's shared memory
+// (one region whose shared address is a multiple of kDecTabAlign).  Every
+// lookup address is "(region | index << 7 | lane bits) + table offset": the
+// index is moved into place with one shift and merged with one mask-or, the
+// table offset is the load's immediate.
+//  * hi pair tables P32, widths 1..3: entry c0 | c1 << w is the fp16 half2
+//    (cb[c0], cb[c1]) (hi parts), one copy per lane at entry * 128 + lane * 4:
+//    a warp-wide 32-bit lookup never has a bank conflict;
+//  * hi|lo pair tables P16, widths 1..4: entry c0 | c1 << w is the 8 bytes
+//    {hi half2, lo half2} of (cb[c0], cb[c1]), one copy per lane pair at
+//    entry * 128 + (lane & 15) * 8: a 64-bit lookup is two conflict-free
+//    half-warp phases;
+//  * hi|lo single-code tables S32, widths 5 and 6: entry c holds the fp16 hi
+//    part (low half) and lo part (high half) of cb[c], at c * 128 + lane * 4;
+//  * shared single-code table SS, widths 1..8 (same entry format), one copy at
+//    kSingleOff(w) + c * 4 (widths 7 and 8, bank conflicts accepted).
+// hi = fp16(cb), lo = fp16(cb - hi).
+constexpr uint32_t kDecTabAlign = 32768;  // P16 width 4: 256 entries << 7
+constexpr uint32_t kTabP16W4 = 0;
+constexpr uint32_t kTabP16W3 = kTabP16W4 + (256u << 7);
+constexpr uint32_t kTabP16W2 = kTabP16W3 + (64u << 7);
+constexpr uint32_t kTabP16W1 = kTabP16W2 + (16u << 7);
+constexpr uint32_t kTabP32W3 = kTabP16W1 + (4u << 7);
+constexpr uint32_t kTabP32W2 = kTabP32W3 + (64u << 7);
+constexpr uint32_t kTabP32W1 = kTabP32W2 + (16u << 7);
+constexpr uint32_t kTabS32W5 = kTabP32W1 + (4u << 7);
+constexpr uint32_t kTabS32W6 = kTabS32W5 + (32u << 7);
+constexpr uint32_t kTabSS = kTabS32W6 + (64u << 7);
+constexpr int kDecodeImageBytes = (int)(kTabSS + 2048u);
+__host__ __device__ constexpr uint32_t kTabP16(int w) {
+  return w == 4 ? kTabP16W4 : (w == 3 ? kTabP16W3 : (w == 2 ? kTabP16W2 : kTabP16W1));
 }
-constexpr uint32_t kSharedSingles = 14336;
+__host__ __device__ constexpr uint32_t kTabP32(int w) {
+  return w == 3 ? kTabP32W3 : (w == 2 ? kTabP32W2 : kTabP32W1);
+}
+__host__ __device__ constexpr uint32_t kTabS32(int w) { return w == 5 ? kTabS32W5 : kTabS32W6; }
 __host__ __device__ constexpr uint32_t kSingleOff(int w) { return 2048u - (8u << w); }
-// regions: pairs w3 [0, 8K), w2 [8K, 10K), w1 [10K, 10.5K); lane singles w4
-// [12K, 14K), w6 [16K, 24K), w5 [24K, 28K); shared singles [14K, 16K)
-static_assert(kPairOff(2) >= kPairOff(3) + (64u << 7) && kPairOff(1) >= kPairOff(2) + (16u << 7) &&
-                  kLaneSingleOff(4) >= kPairOff(1) + (4u << 7) &&
-                  kSharedSingles >= kLaneSingleOff(4) + (16u << 7) &&
-                  kLaneSingleOff(6) >= kSharedSingles + 2048u &&
-                  kLaneSingleOff(5) >= kLaneSingleOff(6) + (64u << 7) &&
-                  (uint32_t)kDecodeImageBytes >= kLaneSingleOff(5) + (32u << 7),
-              "decode table regions overlap");
+static_assert(kDecodeImageBytes % 16 == 0 && kDecodeImageBytes <= 72 * 1024, "decode tables");
+
+// Key rotation of one head for the decode kernel's query rotation
+// ("rotation pack", fp32 words): words [0, 32) hold coord_dim[128] (uint8: the
+// head dim of packed position p's group coordinate p - first(g)), then for
+// every key group g in order its R_m transposed, m x m floats with element
+// (c, r) = R_m[r][c] at word 32 + (sum over earlier groups of m^2) + c * m + r.
+constexpr int kRotPackHeaderWords = 32;
+constexpr int kRotPackMaxWords = kRotPackHeaderWords + kD * kD;
+constexpr size_t kRotPackBytes = (size_t)kRotPackMaxWords * 4;
+
+// Per-head split-merge counters of the decode kernel: [0] second-level
+// ticket, [1, 1 + kMaxMergeGroups) first-level tickets, [kSchedWord] the
+// dynamic tile counter.  Each is returned to 0 by the call that finishes with it.
+constexpr int kSchedWord = 1 + kMaxMergeGroups;
+constexpr int kTicketStride = kSchedWord + 1;
 
 // Code lookup table of the tensor-core quantizer, one part per width w = 1..8.
 // Cell of an fp32 value z: floor(z * inv[w]) + k[w], evaluated as
@@ -139,10 +164,10 @@ struct gtq_plan {
   uint8_t* d_bits;    // [heads][n_blocks]
   gtq::HeadMeta* d_meta;  // [heads]
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
-  float* d_mrow_t;    // [heads][128][128] the same, transposed: [dim][packed position]
+  float* d_rotpack;   // [heads][kRotPackMaxWords] key rotation blocks for the decode kernel
   uint8_t* d_bimg;    // [heads] M_h as the quantizer's tensor-core B operand (64 KB each)
   float* d_partials;  // [heads][kPartialSlots][8][kPartialStride]
-  unsigned* d_tickets;  // [heads][1 + kMaxMergeGroups] arrival counters of the split merge
+  unsigned* d_tickets;  // [heads][kTicketStride] split-merge tickets and the tile counter
   int* d_status;      // device status word
 };
 

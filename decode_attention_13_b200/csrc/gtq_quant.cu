@@ -1,7 +1,7 @@
 // TurboQuant-MSE quantize-pack of keys (Block-GTQ mixed widths) and values
 // (uniform width) into the packed cache ("RoPE-Aware Bit Allocation for
-// KV-Cache Quantization", Abstract: Block-GTQ is "built on TurboQuant-MSE";
-// the page's "packed-cache serving path" stores the codes).
+// KV-Cache Quantization", Abstract: Block-GTQ uses TurboQuant-MSE as its base
+// quantizer, and the page serves decoding from the packed codes).
 //
 // Per token and key group g (width w, m coordinates): n = ||k_g|| (fp64 sum of
 // exact squares, blocks ascending, p0 then p1), y = (sqrt(m)/n) (M_h k)[rows of

@@ -1,8 +1,8 @@
 // Tensor-core quantize-pack (fp16 K/V, head_dim 128): the per-token rotations
 // run as tcgen05 GEMMs with fp32 accumulators in tensor memory ("RoPE-Aware Bit
-// Allocation for KV-Cache Quantization", Abstract: Block-GTQ quantizes keys
-// "built on TurboQuant-MSE", whose coder rotates every normalised vector before
-// scalar Lloyd-Max coding).  Stored values are those of the CUDA-core quantizer
+// Allocation for KV-Cache Quantization", Abstract: Block-GTQ quantizes keys with
+// TurboQuant-MSE as the base quantizer, whose coder rotates every normalised
+// vector before scalar Lloyd-Max coding).  Stored values are those of the CUDA-core quantizer
 // (gtq_quant.cu): per token and key group g, n = ||k_g||, code = number of fp32
 // thresholds below (sqrt(m)/n) (M_h k)_j, fp16(n) stored; values likewise with
 // one group of 128 and R_V.

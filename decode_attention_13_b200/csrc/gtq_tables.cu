@@ -249,23 +249,29 @@ int tables_for(int device, uint64_t seed, Tables* out) {
       llo[lut_base(w) + k] = __double2half(r.c[k] - (double)__half2float(h));
     }
   }
-  // decode lookup-table image (layout: see kPairOff / kLaneSingleOff / kSingleOff)
+  // decode lookup-table image (layout: gtq_internal.h, kTab*)
   std::vector<uint32_t> img(kDecodeImageBytes / 4, 0u);
   auto bits16 = [](__half h) { uint16_t u; std::memcpy(&u, &h, 2); return (uint32_t)u; };
-  auto hilo = [&](int w, int c) {
-    return bits16(lhi[lut_base(w) + c]) | (bits16(llo[lut_base(w) + c]) << 16);
-  };
-  for (int w = 1; w <= 3; ++w)
+  auto hi = [&](int w, int c) { return bits16(lhi[lut_base(w) + c]); };
+  auto lo = [&](int w, int c) { return bits16(llo[lut_base(w) + c]); };
+  for (int w = 1; w <= 4; ++w)
     for (int idx = 0; idx < (1 << (2 * w)); ++idx) {
       const int c0 = idx & ((1 << w) - 1), c1 = idx >> w;
-      const uint32_t v = bits16(lhi[lut_base(w) + c0]) | (bits16(lhi[lut_base(w) + c1]) << 16);
-      for (int lane = 0; lane < 32; ++lane) img[kPairOff(w) / 4 + idx * 32 + lane] = v;
+      const uint32_t vh = hi(w, c0) | (hi(w, c1) << 16), vl = lo(w, c0) | (lo(w, c1) << 16);
+      for (int cp = 0; cp < 16; ++cp) {  // P16: {hi half2, lo half2} per lane pair
+        img[(kTabP16(w) + idx * 128 + cp * 8) / 4] = vh;
+        img[(kTabP16(w) + idx * 128 + cp * 8) / 4 + 1] = vl;
+      }
+      if (w <= 3)
+        for (int lane = 0; lane < 32; ++lane) img[(kTabP32(w) + idx * 128 + lane * 4) / 4] = vh;
     }
-  for (int w = 4; w <= 6; ++w)
+  for (int w = 5; w <= 6; ++w)
     for (int c = 0; c < (1 << w); ++c)
-      for (int lane = 0; lane < 32; ++lane) img[kLaneSingleOff(w) / 4 + c * 32 + lane] = hilo(w, c);
+      for (int lane = 0; lane < 32; ++lane)
+        img[(kTabS32(w) + c * 128 + lane * 4) / 4] = hi(w, c) | (lo(w, c) << 16);
   for (int w = 1; w <= GTQ_MAX_BITS; ++w)
-    for (int c = 0; c < (1 << w); ++c) img[(kSharedSingles + kSingleOff(w)) / 4 + c] = hilo(w, c);
+    for (int c = 0; c < (1 << w); ++c)
+      img[(kTabSS + kSingleOff(w)) / 4 + c] = hi(w, c) | (lo(w, c) << 16);
   Tables t{};
   auto up = [](void** dst, const void* src, size_t bytes) -> cudaError_t {
     cudaError_t e = cudaMalloc(dst, bytes);

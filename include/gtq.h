@@ -2,11 +2,11 @@
  * gtq.h -- C ABI of libgtq: Block-GTQ packed KV cache on NVIDIA B200 (sm_100a).
  *
  * Block-GTQ ("RoPE-Aware Bit Allocation for KV-Cache Quantization", Liang,
- * Zhang, Jia; arXiv 2606.24033, Abstract) quantizes a key cache "built on
- * TurboQuant-MSE": for each layer and KV head it scores every 2-D RoPE block
- * with a label-free energy and "greedily allocates integer bit widths by
- * marginal gain"; the page's "packed-cache serving path" then decodes over the
- * packed cache.  This library implements that hot path:
+ * Zhang, Jia; arXiv 2606.24033, Abstract) quantizes a key cache with
+ * TurboQuant-MSE as the base quantizer: for each layer and KV head it scores
+ * every 2-D RoPE block with an energy that needs no labels and gives out
+ * integer bit widths one bit at a time by marginal gain; decoding then reads
+ * the packed cache directly.  This library implements that hot path:
  *
  *   gtq_alloc_bits     energy of each RoPE block + greedy bit allocation
  *   gtq_quantize_pack  TQ-MSE group coding of K (mixed widths) and V (uniform)
@@ -103,9 +103,8 @@ typedef struct gtq_config {
 } gtq_config;
 
 /*
- * gtq_alloc_bits -- energy pass + greedy allocation (the page's "label-free
- * energy score for each RoPE block" and greedy "integer bit widths by marginal
- * gain", Abstract).
+ * gtq_alloc_bits -- energy pass + greedy allocation (the page's per-block
+ * energy score and its one-bit-at-a-time marginal-gain allocation, Abstract).
  *   cfg        configuration (copied).
  *   k_dev      post-RoPE keys, in_dtype, element (b, h, t, i) at
  *              k_dev + b*k_strides[0] + h*k_strides[1] + t*k_strides[2] + i*k_strides[3]
@@ -153,8 +152,8 @@ GTQ_API int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_d
 
 /*
  * gtq_decode_attn -- fused GQA decode attention of one query token per sequence
- * over the first T tokens of the packed cache (the page's packed-cache serving
- * path).  Scores are taken in each group's rotated basis, softmax is online and
+ * over the first T tokens of the packed cache (the page decodes straight from
+ * the packed cache, Abstract).  Scores are taken in each group's rotated basis, softmax is online and
  * split over the context, P.V accumulates in V's rotated basis and R_V^T is
  * applied once when the splits merge.
  *   packed_dev  cache written by gtq_quantize_pack for tokens [0, T).

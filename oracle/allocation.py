@@ -1,8 +1,9 @@
 """Block-GTQ energy score, greedy bit allocation and block groups (oracle).
 
-"For each layer and KV head, Block-GTQ computes a label-free energy score for
-each RoPE block and greedily allocates integer bit widths by marginal gain"
-("RoPE-Aware Bit Allocation for KV-Cache Quantization", Abstract).
+Per layer and KV head, Block-GTQ scores every RoPE block with an energy that
+needs no labels, then hands out integer bit widths one at a time to the block
+whose next bit gains the most ("RoPE-Aware Bit Allocation for KV-Cache
+Quantization", Abstract).
 
 Readings taken (the page prints no formula):
 

@@ -1,7 +1,7 @@
 """GQA decode attention over Block-GTQ codes (oracle, fp64).
 
-The page describes "a packed-cache serving path" that decodes over the packed
-K/V cache ("RoPE-Aware Bit Allocation for KV-Cache Quantization", Abstract).
+The page reports decoding straight from the packed K/V cache at serving time
+("RoPE-Aware Bit Allocation for KV-Cache Quantization", Abstract).
 The construction read for it: the logit uses the dequantised keys, and since
 every group's rotation is orthogonal it can be taken in the rotated basis,
 

@@ -1,7 +1,7 @@
 """Lloyd-Max scalar quantizer of a standard normal variable (oracle, fp64).
 
-Block-GTQ is "built on TurboQuant-MSE (TQ-MSE)" ("RoPE-Aware Bit Allocation
-for KV-Cache Quantization", Abstract).  TQ-MSE codes each rotated, normalised
+Block-GTQ takes TurboQuant-MSE (TQ-MSE) as its base quantizer ("RoPE-Aware
+Bit Allocation for KV-Cache Quantization", Abstract).  TQ-MSE codes each rotated, normalised
 coordinate with the MSE-optimal (Lloyd-Max) scalar quantizer of N(0, 1), and
 Block-GTQ's marginal gain of one more bit on a block is measured with that
 quantizer's distortion D(b).

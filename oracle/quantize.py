@@ -1,8 +1,8 @@
 """TurboQuant-MSE group coding of keys and values (oracle, fp64).
 
-Block-GTQ quantizes keys "built on TurboQuant-MSE (TQ-MSE)" and compares with
-"uniform TQ-MSE" at matched K/V bit budgets ("RoPE-Aware Bit Allocation for
-KV-Cache Quantization", Abstract).
+Block-GTQ codes keys with TurboQuant-MSE (TQ-MSE) as the base quantizer and is
+compared against TQ-MSE with one width for every block, at the same K/V bit
+budgets ("RoPE-Aware Bit Allocation for KV-Cache Quantization", Abstract).
 
 Construction read for this implementation:
 

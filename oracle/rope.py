@@ -1,8 +1,9 @@
 """RoPE 2-D frequency blocks and the block decomposition of a logit (oracle).
 
-"Under RoPE, however, a key's contribution to a future attention logit
-decomposes into a position-dependent sum over two-dimensional frequency
-blocks" ("RoPE-Aware Bit Allocation for KV-Cache Quantization", Abstract).
+With RoPE, the part of a future attention logit that a key contributes splits
+into a sum of terms, one per two-dimensional frequency block, each depending on
+the relative position ("RoPE-Aware Bit Allocation for KV-Cache Quantization",
+Abstract).
 
 With frequencies w_i = theta**(-2 i / d), i = 0..d/2-1, RoPE rotates the 2-D
 block i of a vector at position p by the angle p * w_i.  For a query at

@@ -1,7 +1,7 @@
 """Seeded orthogonal rotations R_m of TurboQuant-MSE (oracle, fp64).
 
-TQ-MSE ("RoPE-Aware Bit Allocation for KV-Cache Quantization", Abstract: the
-allocator is "built on TurboQuant-MSE") rotates each normalised vector by a
+TQ-MSE (the base quantizer of the allocator in "RoPE-Aware Bit Allocation for
+KV-Cache Quantization", Abstract) rotates each normalised vector by a
 fixed random orthogonal matrix so that every rotated coordinate is close to
 N(0, 1/m), then codes sqrt(m) times each coordinate with the Lloyd-Max
 quantizer of N(0, 1).

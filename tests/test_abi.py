@@ -114,3 +114,15 @@ def test_strerror_names():
     for code in range(-7, 1):
         assert gtq.strerror(code) and gtq.strerror(code) != "unknown error"
     assert gtq.strerror(-99) == "unknown error"
+
+
+def test_noalloc_energy_rejects_head_count_overflow():
+    # batch * n_kv_heads is formed in 64 bits and bounded by the grid limit
+    # (65535) before any device call, so this runs without a GPU
+    lib = gtq.binding._lib
+    st = (ctypes.c_int64 * 4)(0, 0, 128, 1)
+    for batch, hkv in ((65536, 1), (1 << 20, 1 << 12), (2 ** 31 - 1, 2 ** 31 - 1)):
+        cfg = gtq.make_config(batch, hkv, hkv, 3, 3, 64)
+        rc = lib.gtq_block_energy_noalloc(ctypes.byref(cfg), 0x1000, 64, st, 0x1000, None)
+        assert rc == gtq.GTQ_ERR_INVALID
+        assert "65535" in lib.gtq_last_error().decode()

@@ -3,14 +3,21 @@
 For each of the four fp16 workloads (one layer of it: the library's unit), the
 library builds the packed cache of the whole layer (energy, greedy allocation,
 quantize-pack) and decodes it with one gtq_decode_attn call, exactly as the
-benchmark does.  The oracle then checks one sampled KV head in full:
-  * its block energies (fp64, rtol 1e-12) and bit allocation (exact);
-  * the codes and norms of 4096 sampled tokens plus the first and last tile
-    (codes within one level, <= 1e-4 of them off; norms within one fp16 ulp,
-    <= 1e-4 of them off);
-  * the attention output of its query heads, decoded by the oracle from the
-    codes read back out of the library's packed cache (identical packed inputs),
+benchmark does.  The oracle then checks:
+  * every KV head: its block energies (fp64, rtol 1e-12) and its bit
+    allocation (exact, the oracle's greedy on fp64 energies);
+  * four KV heads (first, last, and two others; in the batched workload two of
+    them come from different sequences): the codes and norms of 4096 sampled
+    tokens plus the first and last tile (codes within one level, <= 1e-4 of
+    them off; norms within one fp16 ulp, <= 1e-4 of them off), and the
+    attention output of their query heads, decoded by the oracle from the codes
+    read back out of the library's packed cache (identical packed inputs),
     within 2e-3 relative L2.
+
+Energies for the allocation check are vectorised fp64 sums (pairwise order);
+where the greedy decision is close enough to a tie that a relative change of
+1e-12 in the energies changes it, the head's energies are recomputed with the
+oracle's correctly rounded sums (math.fsum) before the comparison.
 """
 
 import numpy as np
@@ -36,6 +43,64 @@ def _rel_l2(a, b):
     return float(np.linalg.norm(np.asarray(a, np.float64) - b) / np.linalg.norm(b))
 
 
+def _energy_vec(k_head):
+    """E_i of one head from its fp16 keys [T, 128] (HALF pairing), fp64."""
+    kk = k_head.astype(np.float64)
+    sq = np.sum(kk * kk, axis=0)
+    return (sq[:64] + sq[64:]) / kk.shape[0]
+
+
+def _oracle_bits(k_head, kb):
+    e = _energy_vec(k_head)
+    bits = allocation.greedy_bits(e, kb, 128)
+    for f in (1 + 1e-12, 1 - 1e-12):
+        rng = np.random.default_rng(int(f * 1e6))
+        alt = allocation.greedy_bits(e * (1 + (f - 1) * rng.uniform(-1, 1, e.shape)), kb, 128)
+        if not np.array_equal(alt, bits):        # near-tie: use the exact sums
+            e = allocation.block_energy(k_head, 0)
+            return e, allocation.greedy_bits(e, kb, 128)
+    return e, bits
+
+
+def _check_head_codes(head_bytes, bits, kb, vb, T, k_np, v_np, seed):
+    keys, vcodes, vnorm = layout.read_head(head_bytes, bits, kb, vb, T)
+    rng = np.random.default_rng(seed)
+    idx = np.unique(np.concatenate([np.arange(min(64, T)), np.arange(max(0, T - 64), T),
+                                    rng.choice(T, min(T, SAMPLE_TOKENS), replace=False)]))
+    kg = quantize.quantize_keys(k_np[idx], bits, 0)
+    vg = quantize.quantize_values(v_np[idx], vb)
+    by_w = {g.width: g for g in kg}
+    flips = total = nflip = ntot = 0
+    pairs = [(codes[idx], n16[idx], by_w[w].codes, by_w[w].norm16) for (w, codes, n16) in keys]
+    pairs.append((vcodes[idx], vnorm[idx], vg.codes, vg.norm16))
+    for c_got, n_got, c_ref, n_ref in pairs:
+        d = c_got - c_ref
+        assert np.all(np.abs(d) <= 1)
+        flips += int(np.count_nonzero(d))
+        total += d.size
+        nd = n_got.view(np.uint16).astype(np.int64) - n_ref.view(np.uint16).astype(np.int64)
+        assert np.all(np.abs(nd) <= 1)
+        nflip += int(np.count_nonzero(nd))
+        ntot += nd.size
+    assert flips <= CODE_FLIP_MAX * total, (flips, total)
+    assert nflip <= NORM_ULP_MAX * ntot, (nflip, ntot)
+    # the library's own codes as the oracle's decode input
+    coords = {g.width: g.coords for g in kg}
+    ok = [quantize.CodedGroup(w, coords[w], c, n, n.astype(np.float64), False)
+          for (w, c, n) in keys]
+    ov = quantize.CodedGroup(vb, vg.coords, vcodes, vnorm, vnorm.astype(np.float64), False)
+    return ok, ov
+
+
+def _sampled_heads(B, hkv):
+    heads = {(0, 0), (B - 1, hkv - 1)}
+    if B > 1:
+        heads |= {(B // 2, hkv // 2), (1, hkv - 1)}
+    else:
+        heads |= {(0, hkv // 2), (0, max(0, hkv // 2 - 1))}
+    return sorted(heads)
+
+
 @pytest.mark.parametrize("config", [1, 2, 3, 4])
 def test_full_size_layer(config):
     c = synth.CONFIGS[config]
@@ -54,53 +119,23 @@ def test_full_size_layer(config):
     bits_gpu = gtq.gtq_get_bits(plan)
     e_gpu = gtq.gtq_get_energy(plan)
 
-    b, h = B - 1, hkv - 1                                  # the sampled head
-    k_np = k[b, h].cpu().numpy()
-    v_np = v[b, h].cpu().numpy()
-    q_np = q[b, h * gq:(h + 1) * gq].float().cpu().numpy()
-    e = allocation.block_energy(k_np, 0)
-    assert np.allclose(e_gpu[b, h], e, rtol=1e-12, atol=0)
-    bits = allocation.greedy_bits(e, kb, 128)
-    assert np.array_equal(bits_gpu[b, h].astype(np.int64), bits)
+    # every head: energies and allocation
+    for b in range(B):
+        k_b = k[b].cpu().numpy()
+        for h in range(hkv):
+            e, bits = _oracle_bits(k_b[h], kb)
+            assert np.allclose(e_gpu[b, h], e, rtol=1e-12, atol=0), (b, h)
+            assert np.array_equal(bits_gpu[b, h].astype(np.int64), bits), (b, h)
 
+    # sampled heads: codes, norms and the decode output on identical codes
     per = plan.packed_bytes // (B * hkv)
-    head = packed[(b * hkv + h) * per:(b * hkv + h + 1) * per].cpu().numpy()
-    keys, vcodes, vnorm = layout.read_head(head, bits, kb, vb, T)
-
-    # codes and norms of sampled tokens
-    rng = np.random.default_rng(config)
-    idx = np.unique(np.concatenate([np.arange(64), np.arange(T - 64, T),
-                                    rng.choice(T, SAMPLE_TOKENS, replace=False)]))
-    kg = quantize.quantize_keys(k_np[idx], bits, 0)
-    vg = quantize.quantize_values(v_np[idx], vb)
-    by_w = {g.width: g for g in kg}
-    flips = total = nflip = ntot = 0
-    for (w, codes, n16) in keys:
-        d = codes[idx] - by_w[w].codes
-        assert np.all(np.abs(d) <= 1)
-        flips += int(np.count_nonzero(d))
-        total += d.size
-        nd = n16[idx].view(np.uint16).astype(np.int64) - by_w[w].norm16.view(np.uint16).astype(np.int64)
-        assert np.all(np.abs(nd) <= 1)
-        nflip += int(np.count_nonzero(nd))
-        ntot += nd.size
-    d = vcodes[idx] - vg.codes
-    assert np.all(np.abs(d) <= 1)
-    flips += int(np.count_nonzero(d))
-    total += d.size
-    nd = vnorm[idx].view(np.uint16).astype(np.int64) - vg.norm16.view(np.uint16).astype(np.int64)
-    assert np.all(np.abs(nd) <= 1)
-    nflip += int(np.count_nonzero(nd))
-    ntot += nd.size
-    assert flips <= CODE_FLIP_MAX * total, (flips, total)
-    assert nflip <= NORM_ULP_MAX * ntot, (nflip, ntot)
-
-    # the whole head's attention output on the library's own codes
-    oracle_keys = []
-    for (w, codes, n16) in keys:
-        g = by_w[w]
-        oracle_keys.append(quantize.CodedGroup(w, g.coords, codes, n16, n16.astype(np.float64), False))
-    oracle_values = quantize.CodedGroup(vb, vg.coords, vcodes, vnorm, vnorm.astype(np.float64), False)
-    ref = attention.decode_rotated(q_np, oracle_keys, oracle_values)
-    got = out[b, h * gq:(h + 1) * gq].cpu().numpy()
-    assert _rel_l2(got, ref) <= DECODE_REL_L2
+    out_np = out.cpu().numpy()
+    for (b, h) in _sampled_heads(B, hkv):
+        k_np = k[b, h].cpu().numpy()
+        v_np = v[b, h].cpu().numpy()
+        q_np = q[b, h * gq:(h + 1) * gq].float().cpu().numpy()
+        bits = bits_gpu[b, h].astype(np.int64)
+        head = packed[(b * hkv + h) * per:(b * hkv + h + 1) * per].cpu().numpy()
+        ok, ov = _check_head_codes(head, bits, kb, vb, T, k_np, v_np, config * 1000 + b * 10 + h)
+        ref = attention.decode_rotated(q_np, ok, ov)
+        assert _rel_l2(out_np[b, h * gq:(h + 1) * gq], ref) <= DECODE_REL_L2, (b, h)

@@ -280,3 +280,28 @@ def test_greedy_ties_and_cap():
     plan = gtq.gtq_alloc_bits_from_energy(cfg, E)
     assert np.array_equal(gtq.gtq_get_bits(plan)[0, 0].astype(np.int64),
                           allocation.greedy_bits(E[0, 0], 3, 8))
+
+
+def test_config0_as_stated():
+    # the single-head correctness workload exactly as specified: d = 128,
+    # T = 1024, theta = 1e4, one query at position T, decay a = 3 with two
+    # outlier blocks x8, values N(0,1), K3V3, fp32 inputs, seed 0
+    c = synth.CONFIGS[0]
+    assert (c["T"], c["theta"], c["k_bits"], c["v_bits"], c["decay"], c["dtype"]) == \
+        (1024, 1e4, 3, 3, 3.0, "fp32")
+    hd = synth.head(0, T=c["T"], d=128, theta=c["theta"], g_q=1, decay=c["decay"],
+                    dtype=np.float32)
+    case = Case.__new__(Case)
+    case.B, case.hkv, case.gq, case.T, case.kb, case.vb, case.pairing = 1, 1, 1, 1024, 3, 3, 0
+    case.lay = {"k": hd["k"][None, None], "v": hd["v"][None, None], "q": hd["q"][None]}
+    case.cap = case.T
+    case.k = torch.from_numpy(case.lay["k"]).cuda()
+    case.v = torch.from_numpy(case.lay["v"]).cuda()
+    case.q = torch.from_numpy(case.lay["q"]).cuda()
+    case.cfg = gtq.make_config(1, 1, 1, 3, 3, 1024, in_dtype=gtq.DTYPE_FP32)
+    case.plan = gtq.gtq_alloc_bits(case.cfg, case.k, case.T)
+    case.packed = torch.zeros(case.plan.packed_bytes, dtype=torch.uint8, device="cuda")
+    ref = check_case(case)
+    # the quantized decode stays close to unquantized attention on this head
+    exact = attention.attention_exact(hd["q"], hd["k"], hd["v"])
+    assert rel_l2(ref[0], exact) < 0.25
