@@ -36,20 +36,29 @@
 namespace gtq {
 namespace {
 
-constexpr int kPairs = 8;                     // consumer warp pairs (at most)
+// 7 pairs + the producer: at most 4 warps per SM sub-partition, so every warp
+// may hold 128 registers (a 17th warp would cap them at 96)
+constexpr int kPairs = 7;                     // consumer warp pairs (at most)
 constexpr int kCWarps = 2 * kPairs;           // consumer warps (at most)
 constexpr int kThreads = (kCWarps + 1) * 32;  // + the producer warp
-constexpr int kMaxRing = 32;                  // tile stages
+constexpr int kMaxRing = 32;                  // stages
+// A stage holds two adjacent tiles fetched by one bulk copy: the copy engine
+// of an SM takes a roughly fixed time per copy, so 7 KB copies stream at about
+// half the HBM bandwidth and 14 KB copies at nearly all of it (measured).
+constexpr int kTPS = 2;                       // tiles per stage
+constexpr int kSkip = -1;                     // stage tile slot without a tile
+constexpr int kEnd = -2;                      // no tiles left for the pair
+constexpr int kLookahead = 24;                // tiles between the L2 prefetch and the copy
 constexpr int kGrab = 2;                      // tiles per counter grab
+constexpr int kStaticEighths = 7;             // share of a head's tiles dealt out statically
 constexpr uint32_t kTabSharedAddr = 163840;   // shared address of the lookup tables
 constexpr int kSmemBytes = (int)kTabSharedAddr + kDecodeImageBytes;
-constexpr int kPackPrefix = 16384;            // rotation-pack bytes fetched with the metadata
+constexpr int kPackPrefix = 24576;            // rotation-pack bytes fetched with the metadata
 constexpr int kPackArea = (int)((kRotPackBytes + 127) & ~size_t(127));
 constexpr int kWoBytes = kCWarps * 8 * kD * 4;           // warps' o at the merge
 constexpr int kScratchBytes = 2 * 8 * kPartialStride * 4;  // split-merge scratch
 constexpr int kRvOff = (kWoBytes + kScratchBytes + 127) & ~127;
 constexpr int kTailBytes = kRvOff + kD * kD * 4;          // + R_V
-constexpr uint32_t kSuspendHintNs = 1000000;  // mbarrier try_wait suspend-time hint
 constexpr uint64_t kWaitNs = 2000000000ull;    // bound of one wait
 constexpr int64_t kPrefetchBudget = 48ll << 20;  // bytes of L2 prefetch per launch
 static_assert(kTabSharedAddr % kDecTabAlign == 0, "table region alignment");
@@ -74,11 +83,13 @@ struct DecodeArgs {
   int64_t T;
   int64_t n_tiles;    // capacity tiles per head (contiguous layout)
   int tile_bytes;
-  int stride;         // bytes per stage
+  int stride;         // bytes per stage (kTPS tiles)
   int kb;
   int ring;           // stages
   int np;             // consumer warp pairs
   int prefetch;       // tiles this CTA prefetches into L2 before the dependency wait
+  int64_t static_per; // tiles [split * static_per, +static_per) are this CTA's; the rest
+                      // (from splits * static_per on) go out through the tile counter
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -125,20 +136,22 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
   return pol;
 }
 
-// bounded wait on an mbarrier phase; false after about two seconds.  Each try
-// suspends the thread until the phase completes or a time hint expires.
+// bounded wait on an mbarrier phase; false after about two seconds.  try_wait
+// without a suspend-time hint blocks for a short, hardware-chosen time and
+// returns as soon as the phase completes; a hint long enough to matter here
+// woke the waiting producer microseconds late and starved the tile pipeline.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned phase) {
   uint64_t t0 = 0;
   for (unsigned i = 0;; ++i) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
         " selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase), "r"(kSuspendHintNs)
+        : "r"(smem_u32(bar)), "r"(phase)
         : "memory");
     if (ok) return true;
-    if ((i & 15u) == 15u) {
+    if ((i & 63u) == 63u) {
       uint64_t now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0)
@@ -196,9 +209,9 @@ struct DecodeSmem {
   uint64_t pack_bar;            // rest of the rotation pack landed
   uint64_t done_bar;            // query rotation done: the pack's stages may be filled
   uint64_t rv_bar;              // R_V landed
-  uint64_t full[kMaxRing];      // stage holds its tile (or an end marker)
-  uint64_t empty[kMaxRing];     // stage released by both warps of its pair
-  int stage_tile[kMaxRing];
+  uint64_t full[kMaxRing];      // stage holds its tiles (or end markers)
+  uint64_t empty[kMaxRing];     // stage released by the warps of both tile slots
+  int2 stage_tile[kMaxRing];    // tile of each slot, kSkip or kEnd
   float wm[kCWarps][8], wl[kCWarps][8], wsc[kCWarps][8], hm[8], hl[8];
   int flag;
   int failed;
@@ -536,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     mbar_init(&s.rv_bar, 1);
     for (int i = 0; i < S; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 2);
+      mbar_init(&s.empty[i], 2 * kTPS);
     }
     s.failed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -544,20 +557,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     mbar_expect_tx(&s.tab_bar, (unsigned)kDecodeImageBytes);
     bulk_copy(tab, a.dec_image, kDecodeImageBytes, &s.tab_bar);
   }
-  // L2 prefetch of the tiles this CTA will most likely take (the counter hands
-  // tiles out in order, so split k's share is [k P, k P + P)).  A prefetch
+  // L2 prefetch of the first tiles of this CTA's static share.  A prefetch
   // changes no value a later load returns, so it may run before the wait; the
   // sizes read here may be stale, which only changes how much is prefetched.
-  if (producer && a.prefetch > 0) {
+  // One prefetch covers the whole range: the copy engine's time goes by copies.
+  if (producer && lane == 0 && a.prefetch > 0 && !hv.pages) {
     const int64_t Tp = a.seq_lens ? (int64_t)__ldcg(a.seq_lens + b) : a.T;
     const int64_t tiles = (min(max(Tp, (int64_t)0), a.T) + kTile - 1) / kTile;
-    int g = __ldcg(&a.meta[head].n_groups);
-    g = min(max(g, 1), kMaxGroups);
-    const unsigned bytes = (unsigned)min(1024 * (a.kb + VB) + 128 + 128 * g, a.tile_bytes);
-    for (int i = lane; i < a.prefetch; i += 32) {
-      const int64_t t = (int64_t)split * a.prefetch + i;
-      if (t < tiles) prefetch_l2(hv.tile(a.packed, t), bytes);
-    }
+    const int64_t t0 = (int64_t)split * a.static_per;
+    const int64_t n = min((int64_t)a.prefetch, tiles - t0);
+    if (n > 0) prefetch_l2(hv.tile(a.packed, t0), (unsigned)(n * a.tile_bytes));
+    const int64_t dyn0 = (int64_t)nsplit * a.static_per;
+    const int64_t dper = (tiles - dyn0 + nsplit - 1) / nsplit;
+    const int64_t d0 = dyn0 + (int64_t)split * dper, dn = min(dper, tiles - d0);
+    if (dper > 0 && dn > 0) prefetch_l2(hv.tile(a.packed, d0), (unsigned)(dn * a.tile_bytes));
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -580,52 +593,105 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
 
   if (producer) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the schedule (lane 0's counter grabs are broadcast);
+    // lane 0 issues the stage copies, and every lane prefetches the cache lines
+    // of the tiles kLookahead ahead into L2 through the load path, which keeps
+    // HBM busy without holding shared memory or the copy engine.
+    {
       int fills = 0;
-      if (!mbar_wait(&s.meta_bar, 0)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_bar, 0))) {
         failed = true;
       } else {
         const int load_bytes = 1024 * (a.kb + VB) + 128 + 128 * s.meta.n_groups;
         const int pack_lo = area - kPackArea;
         const uint64_t pol = evict_first_policy();
         unsigned* ctr = head_tickets + kSchedWord;
+        // static share first; the counter's grabs are issued ahead of use, so
+        // their round trip never holds up a load
+        const int64_t st0 = min((int64_t)split * a.static_per, tiles_T);
+        const int64_t st1 = min(st0 + a.static_per, tiles_T);
+        const int64_t dyn0 = (int64_t)nsplit * a.static_per;
+        const int64_t pf_done = st0 + a.prefetch;  // prefetched before the wait
+        int64_t snext = st0;
         bool setup_ok = false, exhausted = false;
-        int cur = (int)atomicAdd(ctr, (unsigned)kGrab), used = 0;
-        int nxt = (int)atomicAdd(ctr, (unsigned)kGrab);
+        auto grab = [&]() -> int {
+          int v = 0;
+          if (lane == 0) v = (int)atomicAdd(ctr, (unsigned)kGrab);
+          return __shfl_sync(0xffffffffu, v, 0);
+        };
+        int g0 = grab(), g1 = grab();
+        int used = 0;
+        auto next_tile = [&]() -> int64_t {
+          if (snext < st1) return snext++;
+          if (exhausted) return -1;
+          if (used == kGrab) {
+            g0 = g1;
+            used = 0;
+            if (dyn0 + g0 < tiles_T) g1 = grab();
+          }
+          const int64_t t = dyn0 + g0 + used++;
+          if (t >= tiles_T) {
+            exhausted = true;
+            return -1;
+          }
+          return t;
+        };
+        const int lines = a.tile_bytes >> 7;
+        auto lookahead = [&](int64_t t) {  // static-share tiles only
+          const int64_t tp = t + kLookahead;
+          if (t < 0 || tp < pf_done || tp >= st1 || hv.pages) return;
+          const uint8_t* base = hv.tile(a.packed, tp);
+          for (int l = lane; l < lines; l += 32)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(base + ((size_t)l << 7)));
+        };
+        int64_t pending = next_tile();
         int ends = 0, slot = 0, round = 0;
         for (;; ++fills) {
-          if (round > 0 && !mbar_wait(&s.empty[slot], (unsigned)(round - 1) & 1u)) {
+          if (round > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(&s.empty[slot], (unsigned)(round - 1) & 1u))) {
             failed = true;
             break;
           }
           if (!setup_ok && (slot + 1) * a.stride > pack_lo) {
-            if (!mbar_wait(&s.done_bar, 0)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.done_bar, 0))) {
               failed = true;
               break;
             }
             setup_ok = true;
           }
-          int64_t t = -1;
-          if (!exhausted) {
-            if (used == kGrab) {
-              cur = nxt;
-              used = 0;
-              if ((int64_t)cur < tiles_T) nxt = (int)atomicAdd(ctr, (unsigned)kGrab);
+          uint8_t* dst = stages + (size_t)slot * a.stride;
+          if (pending >= 0) {
+            const int64_t t0 = pending;
+            pending = next_tile();
+            int64_t t1 = kSkip;
+            if (pending == t0 + 1) {
+              t1 = pending;
+              pending = next_tile();
             }
-            t = (int64_t)cur + used++;
-            if (t >= tiles_T) {
-              t = -1;
-              exhausted = true;
+            if (lane == 0) {
+              s.stage_tile[slot] = make_int2((int)t0, (int)t1);
+              if (t1 >= 0 && !hv.pages) {  // adjacent tiles: one copy
+                mbar_expect_tx(&s.full[slot], (unsigned)(a.tile_bytes + load_bytes));
+                bulk_copy_hint(dst, hv.tile(a.packed, t0), (unsigned)(a.tile_bytes + load_bytes),
+                               &s.full[slot], pol);
+              } else {
+                mbar_expect_tx(&s.full[slot], (unsigned)(t1 >= 0 ? 2 * load_bytes : load_bytes));
+                bulk_copy_hint(dst, hv.tile(a.packed, t0), (unsigned)load_bytes, &s.full[slot], pol);
+                if (t1 >= 0)
+                  bulk_copy_hint(dst + a.tile_bytes, hv.tile(a.packed, t1), (unsigned)load_bytes,
+                                 &s.full[slot], pol);
+              }
             }
-          }
-          s.stage_tile[slot] = (int)t;
-          if (t >= 0) {
-            mbar_expect_tx(&s.full[slot], (unsigned)load_bytes);
-            bulk_copy_hint(stages + (size_t)slot * a.stride, hv.tile(a.packed, t),
-                           (unsigned)load_bytes, &s.full[slot], pol);
+            lookahead(t0);
+            lookahead(t1);
           } else {
-            mbar_arrive(&s.full[slot]);
-            if (++ends == np) {
+            // end markers: every pair meets one as its next tile slot
+            if (lane == 0) {
+              s.stage_tile[slot] = make_int2(kEnd, kEnd);
+              mbar_arrive(&s.full[slot]);
+            }
+            ends += kTPS;
+            if (ends >= np) {
               ++fills;
               break;
             }
@@ -635,15 +701,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             ++round;
           }
         }
-        asm volatile("" ::"r"(nxt));  // every grab has returned before the CTA moves on
+        asm volatile("" ::"r"(g0), "r"(g1));  // every grab has returned before the CTA moves on
       }
       // drain: no bulk copy into this CTA's shared memory may outlive the loop
-      const int n_used = min(fills, S);
-      for (int sl = 0; sl < n_used; ++sl) {
-        const int last = sl + ((fills - 1 - sl) / S) * S;  // last fill index of the slot
-        mbar_wait(&s.full[sl], (unsigned)(last / S) & 1u);
+      if (lane == 0) {
+        const int n_used = min(fills, S);
+        for (int sl = 0; sl < n_used; ++sl) {
+          const int last = sl + ((fills - 1 - sl) / S) * S;  // last fill index of the slot
+          mbar_wait(&s.full[sl], (unsigned)(last / S) & 1u);
+        }
       }
-      if (failed) s.failed = 1;
+      if (failed && lane == 0) s.failed = 1;
     }
   } else {
     // ------------------------------------------------------------ consumers
@@ -750,7 +818,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     // lane portion of slot t: 16W bits at byte 16W t + 2W g; this warp's half: + W wh
     const int lane_kunit = 16 * t + 2 * g + wh;  // times W
 
-    int slot = pair, round = 0;
+    // tile slot j = pair + k np of the stage sequence: stage j / kTPS, slot j % kTPS
+    int j = pair, fi = pair / kTPS, slot = fi % S, round = fi / S;
     // a timeout seen by any lane stops the whole warp (the loop body is warp-wide)
     failed = __any_sync(0xffffffffu, failed);
     while (!failed) {
@@ -758,9 +827,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         failed = true;
         break;
       }
-      const int tile_idx = s.stage_tile[slot];
-      if (tile_idx < 0) break;
-      const uint8_t* tl = stages + (size_t)slot * a.stride;
+      const int2 st2 = s.stage_tile[slot];
+      const int jk = j % kTPS;
+      const int tile_idx = jk ? st2.y : st2.x;
+      if (tile_idx == kEnd) break;
+      auto advance = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[slot]);
+        j += np;
+        const int nfi = j / kTPS;
+        slot += nfi - fi;
+        fi = nfi;
+        while (slot >= S) {
+          slot -= S;
+          ++round;
+        }
+      };
+      if (tile_idx == kSkip) {
+        advance();
+        continue;
+      }
+      const uint8_t* tl = stages + (size_t)slot * a.stride + (size_t)jk * a.tile_bytes;
 
       // ------------------------------------------------------------ scores
       float S_[2][4];
@@ -864,13 +951,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       for (int i = 0; i < 8; ++i)
         value_tile<VB>(vcodes + ((i * 8 + g) * 4 + t) * VB * 4, wh, tb, PB, O[i]);
       // ---------------------------------------------------- release the stage
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.empty[slot]);
-      slot += np;
-      if (slot >= S) {
-        slot -= S;
-        ++round;
-      }
+      advance();
     }
     if (failed && lane == 0) s.failed = 1;
     // lanes' partial l over their tokens
@@ -905,13 +986,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       s.wl[warp][2 * t] = lrun[0];
       s.wl[warp][2 * t + 1] = lrun[1];
     }
+    // [warp][dim][head]: a lane's two heads are adjacent (one 8-byte store), and
+    // a half-warp's stores cover all 32 banks once
     float* o = wo + warp * 8 * kD;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      o[(2 * t) * kD + 16 * i + g] = O[i][0];
-      o[(2 * t + 1) * kD + 16 * i + g] = O[i][1];
-      o[(2 * t) * kD + 16 * i + g + 8] = O[i][2];
-      o[(2 * t + 1) * kD + 16 * i + g + 8] = O[i][3];
+      *reinterpret_cast<float2*>(o + (16 * i + g) * 8 + 2 * t) = make_float2(O[i][0], O[i][1]);
+      *reinterpret_cast<float2*>(o + (16 * i + g + 8) * 8 + 2 * t) = make_float2(O[i][2], O[i][3]);
     }
   }
   __syncthreads();
@@ -934,9 +1015,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   // this CTA's (m, l, o_rot): the output itself with a single split, else its
   // partial in global memory
   for (int idx = tid; idx < 8 * kD; idx += blockDim.x) {
-    const int hh = idx >> 7, d = idx & (kD - 1);
+    const int hh = idx & 7, d = idx >> 3;
     float v = 0.f;
-    for (int w = 0; w < ncw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * 8 + hh) * kD + d], v);
+    for (int w = 0; w < ncw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * kD + d) * 8 + hh], v);
     if (nsplit == 1) {
       s.qa[hh][d] = s.hl[hh] > 0.f ? v / s.hl[hh] : 0.f;
     } else {
@@ -991,20 +1072,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     if (tid == 0) atomicOr(a.status, kStatusTimeout);
     return;
   }
-  // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r]
-  float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
-  for (int idx = tid; idx < 8 * (kD / 2); idx += blockDim.x) {
-    const int hh = idx / (kD / 2), dd = 2 * (idx % (kD / 2));
-    if (hh >= a.gq) continue;
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-    for (int r = 0; r < kD; ++r) {
-      const float2 w = *reinterpret_cast<const float2*>(rv + r * kD + dd);
-      const float o = s.qa[hh][r];
-      acc0 = fmaf(w.x, o, acc0);
-      acc1 = fmaf(w.y, o, acc1);
+  // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r]: thread = (dd pair, 16 rows r of
+  // one r-group); o_rot^T in qb so that a warp reads its 8 heads of row r as two
+  // broadcasts; the 8 r-groups' partial sums are added through shared memory
+  {
+    float(*oT)[8] = reinterpret_cast<float(*)[8]>(&s.qb[0][0]);  // [r][head]
+    for (int i = tid; i < 8 * kD; i += blockDim.x) oT[i >> 3][i & 7] = s.qa[i & 7][i >> 3];
+    __syncthreads();
+    float* red = wo;  // [r-group][head][dim]
+    for (int task = tid; task < 512; task += blockDim.x) {
+      const int dd = 2 * (task & 63), rg = task >> 6;
+      float acc[8][2];
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
+#pragma unroll 4
+      for (int r = 16 * rg; r < 16 * rg + 16; ++r) {
+        const float2 w = *reinterpret_cast<const float2*>(rv + r * kD + dd);
+        const float4 oa = *reinterpret_cast<const float4*>(&oT[r][0]);
+        const float4 ob = *reinterpret_cast<const float4*>(&oT[r][4]);
+        const float ov[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) {
+          acc[hh][0] = fmaf(w.x, ov[hh], acc[hh][0]);
+          acc[hh][1] = fmaf(w.y, ov[hh], acc[hh][1]);
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh)
+        *reinterpret_cast<float2*>(red + (rg * 8 + hh) * kD + dd) = make_float2(acc[hh][0], acc[hh][1]);
     }
-    *reinterpret_cast<float2*>(out_head + hh * kD + dd) = make_float2(acc0, acc1);
+    __syncthreads();
+    float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
+    for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
+      const int hh = idx >> 7, dd = idx & (kD - 1);
+      float v = 0.f;
+#pragma unroll
+      for (int rg = 0; rg < 8; ++rg) v += red[(rg * 8 + hh) * kD + dd];
+      out_head[idx] = v;
+    }
   }
 }
 
@@ -1049,7 +1154,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.n_tiles = p->n_tiles;
   a.tile_bytes = (int)p->tile_bytes;
   a.kb = p->cfg.k_bits;
-  a.stride = (int)((p->tile_bytes + 127) & ~size_t(127));
+  a.stride = (int)((kTPS * p->tile_bytes + 127) & ~size_t(127));
   int dev_smem = 0;
   cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
   if (dev_smem < kSmemBytes) return cudaErrorInvalidValue;
@@ -1059,7 +1164,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   if (area < kTailBytes || area < kPackArea + a.stride) return cudaErrorInvalidValue;
   const int ring = std::min(kMaxRing, area / a.stride);
   if (ring < 2) return cudaErrorInvalidValue;
-  const int np = std::max(1, std::min(kPairs, ring / 2));
+  const int np = std::max(1, std::min(kPairs, ring * kTPS / 2));
   a.ring = ring;
   a.np = np;
   const int64_t tiles_T = (T + kTile - 1) / kTile;
@@ -1069,9 +1174,9 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
                                 : std::max(1, p->n_sms / p->n_heads);
   splits = (int)std::min<int64_t>(splits, std::max<int64_t>(1, tiles_T));
   splits = std::max(1, std::min(splits, kMaxSplits));
-  const int64_t per = (tiles_T + splits - 1) / splits;
+  a.static_per = tiles_T * kStaticEighths / 8 / splits;
   const int64_t budget = kPrefetchBudget / ((int64_t)p->n_heads * splits * a.tile_bytes);
-  a.prefetch = (int)std::max<int64_t>(0, std::min<int64_t>(per, budget));
+  a.prefetch = (int)std::max<int64_t>(0, std::min<int64_t>(a.static_per, budget));
   cudaError_t e = cudaErrorInvalidValue;
   const dim3 grid((unsigned)p->n_heads, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));
   switch (p->cfg.v_bits) {
