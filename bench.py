@@ -39,7 +39,7 @@ L2_BYTES = 126 * 2 ** 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=2)
@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's context length (overhead studies only)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the per-config and peak-memory blocks (headline workload only)")
     return ap.parse_args()
 
 
@@ -125,6 +127,18 @@ def profile_traffic(kernel_src):
     return float(t.group(1))
 
 
+def workload_config(cfgd, world):
+    """The `config` object of both arms' JSON lines (identical keys)."""
+    step_bytes = cfgd["layers"] * cfgd["B"] * cfgd["h_kv"] * cfgd["T"] * packed_bytes_per_token_head(
+        cfgd["k_bits"], cfgd["v_bits"], 6)
+    return {"workload": cfgd["name"], "layers": cfgd["layers"], "batch": cfgd["B"],
+            "q_heads": cfgd["h_q"], "kv_heads": cfgd["h_kv"], "seq_len": cfgd["T"],
+            "k_bits": cfgd["k_bits"], "v_bits": cfgd["v_bits"],
+            "parallelism": "replicas" if world == 1 else "dp%d (independent sequences)" % world,
+            "l2": "cold: about %.0f MB of packed cache per step > 126 MB L2, layers read in turn"
+                  % (step_bytes / 1e6)}
+
+
 # ------------------------------------------------------------ multi-rank
 def max_over_ranks(value, world, device=None):
     """The largest `value` over all ranks (the job's time is its slowest rank's)."""
@@ -167,56 +181,250 @@ def oracle_threads():
         return 1
 
 
-def oracle_decode_sample(cfgd, pool, seconds):
-    """Time the fp64 oracle's decode of whole KV heads from `pool` until
-    `seconds` elapse; returns (GB/s of packed cache, heads decoded, seconds)."""
+def _head_slice(kg, vg, n):
+    """The first n cached tokens of a coded head (the oracle's data classes)."""
+    import dataclasses
+
+    cut = lambda g: dataclasses.replace(g, codes=g.codes[:n], norm16=g.norm16[:n],
+                                        norm64=g.norm64[:n])
+    return [cut(g) for g in kg], cut(vg)
+
+
+def oracle_decode_sample(cfgd, pool, seconds, tokens=None):
+    """Time the fp64 oracle's decode of KV heads from `pool` until `seconds`
+    elapse (at least one); each decode covers the first `tokens` cached tokens
+    of a head (all T by default).  Returns (GB/s of packed cache, heads decoded,
+    seconds, tokens per decode)."""
     from oracle import attention
 
     T, kb, vb = cfgd["T"], cfgd["k_bits"], cfgd["v_bits"]
+    n = T if tokens is None else max(1, min(T, int(tokens)))
     heads, nbytes, spent = 0, 0.0, 0.0
     while spent < seconds or heads == 0:
         q, kg, vg = pool[heads % len(pool)]
+        if n < T:
+            kg, vg = _head_slice(kg, vg, n)
         t0 = time.perf_counter()
         attention.decode_rotated(q, kg, vg)
         spent += time.perf_counter() - t0
-        nbytes += T * packed_bytes_per_token_head(kb, vb, len(kg))
+        nbytes += n * packed_bytes_per_token_head(kb, vb, len(kg))
         heads += 1
-    return nbytes / spent / 1e9, heads, spent
+    return nbytes / spent / 1e9, heads, spent, n
 
 
 def run_reference(args, rank, world):
     from decode_attention_13_b200 import synth
 
-    cfgd = synth.CONFIGS[args.config]
+    cfgd = dict(synth.CONFIGS[args.config], index=args.config)
     if rank != 0:
         return
     pool = oracle_pool(cfgd)
     threads = oracle_threads()
+    # each step decodes a token slice of one head, sized so that the K steps
+    # take about --cpu-seconds together (a bounded sample of the same work)
     per_step = args.cpu_seconds / max(1, args.steps)
+    _, _, spent, _ = oracle_decode_sample(cfgd, pool, 0.0, tokens=8192)
+    tokens = max(1024, int(8192 * per_step / max(spent, 1e-6)))
     for _ in range(args.warmup):
-        oracle_decode_sample(cfgd, pool, 0.0)
+        oracle_decode_sample(cfgd, pool, 0.0, tokens=tokens)
     vals, heads_total, spent_total = [], 0, 0.0
     for _ in range(args.steps):
-        v, h, s = oracle_decode_sample(cfgd, pool, per_step)
+        v, h, s, n = oracle_decode_sample(cfgd, pool, 0.0, tokens=tokens)
         vals.append(v)
         heads_total += h
         spent_total += s
     value = statistics.mean(vals)
-    sample = ("oracle decode of %d whole KV heads (T=%d, G=%d query heads each) of the %s "
-              "workload; one bounded sample per step" % (heads_total, cfgd["T"],
-                                                         cfgd["h_q"] // cfgd["h_kv"], cfgd["name"]))
+    sample = ("oracle decode of the first %d cached tokens of a KV head (of T=%d, G=%d query "
+              "heads), %d times, from the %s workload; one decode per step"
+              % (min(tokens, cfgd["T"]), cfgd["T"], cfgd["h_q"] // cfgd["h_kv"], heads_total,
+                 cfgd["name"]))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
         "ms_per_step": 1e3 * spent_total / max(1, args.steps), "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfgd["name"], "layers": cfgd["layers"], "batch": cfgd["B"],
-                   "q_heads": cfgd["h_q"], "kv_heads": cfgd["h_kv"], "seq_len": cfgd["T"],
-                   "k_bits": cfgd["k_bits"], "v_bits": cfgd["v_bits"]},
+        "config": workload_config(cfgd, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def build_workload(cfgd, rank, dev, stream):
+    """Every layer's plan and packed cache (energy, greedy allocation,
+    quantize-pack by the library), its queries and output buffers."""
+    import torch
+
+    import decode_attention_13_b200 as gtq
+    from decode_attention_13_b200 import synth
+
+    L, B, hq, hkv, T = cfgd["layers"], cfgd["B"], cfgd["h_q"], cfgd["h_kv"], cfgd["T"]
+    kb, vb, gq = cfgd["k_bits"], cfgd["v_bits"], cfgd["h_q"] // cfgd["h_kv"]
+    w = {"plans": [], "packed": [], "qs": [], "outs": [], "kv": []}
+    for layer in range(L):
+        k, v, q = synth.layer_torch(rank_seed(cfgd["index"], rank, layer), B, hkv, gq, T,
+                                    theta=cfgd["theta"], decay=cfgd["decay"], device=dev)
+        cfg = gtq.make_config(B, hq, hkv, kb, vb, T)
+        with torch.cuda.stream(stream):
+            plan = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
+            buf = torch.empty(plan.packed_bytes, dtype=torch.uint8, device=dev)
+            gtq.gtq_quantize_pack(plan, k, v, 0, T, buf, stream=stream)
+        w["plans"].append(plan)
+        w["packed"].append(buf)
+        w["qs"].append(q)
+        w["outs"].append(torch.empty((B, hq, 128), dtype=torch.float32, device=dev))
+        w["kv"].append((k, v))
+    stream.synchronize()
+    for p in w["plans"]:
+        rc = gtq.gtq_status(p)
+        if rc != gtq.GTQ_OK:
+            raise RuntimeError("status after quantize: " + gtq.strerror(rc))
+    g_k = []  # nonzero-width key groups of every head (norms read per token)
+    for p in w["plans"]:
+        bits = gtq.gtq_get_bits(p)
+        g_k.append([[len(set(int(x) for x in bits[b, h] if x > 0)) for h in range(hkv)]
+                    for b in range(B)])
+    w["step_bytes"] = float(sum(T * packed_bytes_per_token_head(kb, vb, g_k[l][b][h])
+                                for l in range(L) for b in range(B) for h in range(hkv)))
+    w["fp16_bytes"] = float(L * B * hkv * T * 2 * 128 * 2)
+    return w
+
+
+def time_quantize(cfgd, w, stream):
+    """CUDA-event time of one quantize-pack of every layer (ms) and its bytes."""
+    import torch
+
+    import decode_attention_13_b200 as gtq
+
+    T = cfgd["T"]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for layer, (k, v) in enumerate(w["kv"]):
+            gtq.gtq_quantize_pack(w["plans"][layer], k, v, 0, T, w["packed"][layer], stream=stream)
+        ev1.record(stream)
+    stream.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    nbytes = float(cfgd["layers"] * cfgd["B"] * cfgd["h_kv"] * T * 512) + w["step_bytes"]
+    return ms, nbytes
+
+
+def decode_graph(cfgd, w, stream):
+    """The decode step (one gtq_decode_attn per layer) captured in a CUDA graph."""
+    import torch
+
+    import decode_attention_13_b200 as gtq
+
+    T = cfgd["T"]
+
+    def step():
+        for layer in range(cfgd["layers"]):
+            gtq.gtq_decode_attn(w["plans"][layer], w["packed"][layer], T, w["qs"][layer],
+                                w["outs"][layer], stream=stream)
+
+    for _ in range(2):
+        with torch.cuda.stream(stream):
+            step()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    stream.synchronize()
+    return graph, step
+
+
+def time_graph(graph, steps, warmup, stream, barrier=lambda: None):
+    import torch
+
+    for _ in range(max(3, warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return t0.elapsed_time(t1) / steps
+
+
+def per_config_line(cfgd, rank, dev, stream, hbm, steps):
+    """Decode and quantize-pack of one more workload, for the per_config block."""
+    import torch
+
+    w = build_workload(cfgd, rank, dev, stream)
+    q_ms, q_bytes = time_quantize(cfgd, w, stream)
+    graph, _ = decode_graph(cfgd, w, stream)
+    ms = time_graph(graph, steps, 3, stream)
+    gbs = w["step_bytes"] / (ms * 1e-3) / 1e9
+    out = {"workload": cfgd["name"], "decode_ms_per_step": ms, "decode_gbs": gbs,
+           "decode_frac": gbs / hbm, "ctx_tokens_per_s": cfgd["B"] * cfgd["T"] / (ms * 1e-3),
+           "bytes_per_step": w["step_bytes"], "quantize_pack_ms": q_ms,
+           "quantize_pack_gbs": q_bytes / (q_ms * 1e-3) / 1e9,
+           "quantize_pack_frac": q_bytes / (q_ms * 1e-3) / 1e9 / hbm, "timed_steps": steps}
+    del graph, w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def memory_report(cfgd, rank, dev, stream, seq_lens=(131072, 262144, 524288)):
+    """Peak device memory of the packed-cache serving state of the stack at
+    several context lengths: every layer's plan and packed cache built layer by
+    layer (one layer's fp16 K/V alive at a time), then one decode step; against
+    the size of the same cache in fp16."""
+    import torch
+
+    import decode_attention_13_b200 as gtq
+    from decode_attention_13_b200 import synth
+
+    L, B, hq, hkv = cfgd["layers"], cfgd["B"], cfgd["h_q"], cfgd["h_kv"]
+    kb, vb, gq = cfgd["k_bits"], cfgd["v_bits"], cfgd["h_q"] // cfgd["h_kv"]
+    rows = []
+    for T in seq_lens:
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        plans, packed, qs, outs, plan_bytes = [], [], [], [], 0
+        for layer in range(L):
+            k, v, q = synth.layer_torch((cfgd["index"], rank, layer), B, hkv, gq, T,
+                                        theta=cfgd["theta"], decay=cfgd["decay"], device=dev)
+            cfg = gtq.make_config(B, hq, hkv, kb, vb, T)
+            with torch.cuda.stream(stream):
+                plan = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
+                buf = torch.empty(plan.packed_bytes, dtype=torch.uint8, device=dev)
+                gtq.gtq_quantize_pack(plan, k, v, 0, T, buf, stream=stream)
+            stream.synchronize()
+            plan_bytes += gtq.gtq_plan_device_bytes(plan)
+            plans.append(plan)
+            packed.append(buf)
+            qs.append(q)
+            outs.append(torch.empty((B, hq, 128), dtype=torch.float32, device=dev))
+            del k, v
+        with torch.cuda.stream(stream):
+            for layer in range(L):
+                gtq.gtq_decode_attn(plans[layer], packed[layer], T, qs[layer], outs[layer],
+                                    stream=stream)
+        stream.synchronize()
+        peak = torch.cuda.max_memory_allocated(dev) - base + plan_bytes
+        resident = sum(b.numel() for b in packed) + plan_bytes
+        fp16 = L * B * hkv * T * 2 * 128 * 2
+        rows.append({"seq_len": T, "peak_bytes": int(peak), "resident_cache_bytes": int(resident),
+                     "fp16_cache_bytes": int(fp16), "fp16_over_resident": fp16 / resident})
+        del plans, packed, qs, outs
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return {"workload": cfgd["name"] + " (context varied)", "rows": rows,
+            "how": "torch.cuda.max_memory_allocated over building the stack layer by layer "
+                   "(one layer's fp16 K/V alive at a time) and one decode step, plus the plans' "
+                   "own device memory (gtq_plan_device_bytes); fp16 = the same K/V cache in fp16; "
+                   "no model weights are involved"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -227,97 +435,55 @@ def run_ours(args, rank, world):
     import decode_attention_13_b200 as gtq
     from decode_attention_13_b200 import synth
 
-    cfgd = dict(synth.CONFIGS[args.config])
+    cfgd = dict(synth.CONFIGS[args.config], index=args.config)
     if args.seq_len:
         cfgd["T"] = args.seq_len
         cfgd["name"] += " (context overridden to %d)" % args.seq_len
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     L, B, hq, hkv, T = cfgd["layers"], cfgd["B"], cfgd["h_q"], cfgd["h_kv"], cfgd["T"]
-    kb, vb, gq = cfgd["k_bits"], cfgd["v_bits"], cfgd["h_q"] // cfgd["h_kv"]
     assert cfgd["dtype"] == "fp16"
     stream = torch.cuda.Stream(device=dev)
-
-    # ---- build every layer's packed cache (energy, greedy, quantize-pack)
-    plans, packed, qs, outs, kv = [], [], [], [], []
-    for layer in range(L):
-        k, v, q = synth.layer_torch(rank_seed(args.config, rank, layer), B, hkv, gq, T,
-                                    theta=cfgd["theta"], decay=cfgd["decay"], device=dev)
-        cfg = gtq.make_config(B, hq, hkv, kb, vb, T)
-        with torch.cuda.stream(stream):
-            plan = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
-            buf = torch.empty(plan.packed_bytes, dtype=torch.uint8, device=dev)
-            gtq.gtq_quantize_pack(plan, k, v, 0, T, buf, stream=stream)
-        plans.append(plan)
-        packed.append(buf)
-        qs.append(q)
-        outs.append(torch.empty((B, hq, 128), dtype=torch.float32, device=dev))
-        kv.append((k, v))
-    stream.synchronize()
-    for p in plans:
-        rc = gtq.gtq_status(p)
-        if rc != gtq.GTQ_OK:
-            raise RuntimeError("status after quantize: " + gtq.strerror(rc))
-    g_k = []  # nonzero-width key groups of every head (norms read per token)
-    for p in plans:
-        bits = gtq.gtq_get_bits(p)
-        g_k.append([[len(set(int(x) for x in bits[b, h] if x > 0)) for h in range(hkv)]
-                    for b in range(B)])
-    bytes_per_layer = [sum(T * packed_bytes_per_token_head(kb, vb, g_k[l][b][h])
-                           for b in range(B) for h in range(hkv)) for l in range(L)]
-    step_bytes = float(sum(bytes_per_layer))
-
-    # ---- prefill timing: quantize-pack of every layer (A3-A6)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for layer in range(L):
-            k, v = kv[layer]
-            gtq.gtq_quantize_pack(plans[layer], k, v, 0, T, packed[layer], stream=stream)
-        ev1.record(stream)
-    stream.synchronize()
-    quant_ms = ev0.elapsed_time(ev1)
-    quant_bytes = float(L * B * hkv * T * 512) + step_bytes
-
-    # ---- the decode step, captured in a CUDA graph
-    def step():
-        for layer in range(L):
-            gtq.gtq_decode_attn(plans[layer], packed[layer], T, qs[layer], outs[layer],
-                                stream=stream)
-
-    for _ in range(2):
-        with torch.cuda.stream(stream):
-            step()
-    stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
-    stream.synchronize()
+    hbm, peak_kind = peaks()
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
+    w = build_workload(cfgd, rank, dev, stream)
+    step_bytes = w["step_bytes"]
+    # ---- prefill timing: quantize-pack of every layer (A3-A6)
+    quant_ms, quant_bytes = time_quantize(cfgd, w, stream)
+
+    # ---- decode-time append: one new token into every layer's packed cache
+    # (the allocation stays the one computed at prefill), captured in a graph
+    def append_step():
+        for layer, (k, v) in enumerate(w["kv"]):
+            gtq.gtq_quantize_pack(w["plans"][layer], k, v, T - 1, 1, w["packed"][layer],
+                                  stream=stream)
+
+    with torch.cuda.stream(stream):
+        append_step()
+    stream.synchronize()
+    agraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(agraph, stream=stream):
+        append_step()
+    append_ms = time_graph(agraph, 50, 3, stream)
+    del agraph
+
+    # ---- the decode step, captured in a CUDA graph (only decode_kernel runs in it)
+    graph, step = decode_graph(cfgd, w, stream)
+    clocks = ClockSampler(dev.index)
     for _ in range(max(3, args.warmup)):
         graph.replay()
     torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    ms_local = time_graph(graph, args.steps, 0, stream, barrier)
     clk = clocks.stop()
-    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    ms = max_over_ranks(ms_local, world, dev)
 
-    # ---- per-call timing of gtq_decode_attn (roofline of the decode kernel)
+    # ---- latency of one eager gtq_decode_attn call (events around each call)
     call_ms = []
     with torch.cuda.stream(stream):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -326,16 +492,15 @@ def run_ours(args, rank, world):
             for layer in range(L):
                 a, b = evs[layer]
                 a.record(stream)
-                gtq.gtq_decode_attn(plans[layer], packed[layer], T, qs[layer], outs[layer],
-                                    stream=stream)
+                gtq.gtq_decode_attn(w["plans"][layer], w["packed"][layer], T, w["qs"][layer],
+                                    w["outs"][layer], stream=stream)
                 b.record(stream)
             stream.synchronize()
             call_ms.append([a.elapsed_time(b) for a, b in evs])
-    per_call_ms = statistics.mean(call_ms[-1])
-    per_call_bytes = step_bytes / L
+    eager_call_ms = statistics.mean(call_ms[-1])
 
     # ---- end to end through the ABI with host buffers
-    q_host = torch.stack(qs).cpu().pin_memory()
+    q_host = torch.stack(w["qs"]).cpu().pin_memory()
     out_host = torch.empty((L, B, hq, 128), dtype=torch.float32).pin_memory()
     q_dev = torch.empty_like(q_host, device=dev)
     out_dev = torch.empty((L, B, hq, 128), dtype=torch.float32, device=dev)
@@ -343,10 +508,11 @@ def run_ours(args, rank, world):
     def e2e_step():
         q_dev.copy_(q_host, non_blocking=True)
         for layer in range(L):
-            gtq.gtq_decode_attn(plans[layer], packed[layer], T, q_dev[layer], out_dev[layer],
-                                stream=stream)
+            gtq.gtq_decode_attn(w["plans"][layer], w["packed"][layer], T, q_dev[layer],
+                                out_dev[layer], stream=stream)
         out_host.copy_(out_dev, non_blocking=True)
 
+    e2e_steps = max(20, min(args.steps, 200))
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             e2e_step()
@@ -355,25 +521,41 @@ def run_ours(args, rank, world):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(e2e_steps):
             e2e_step()
         e1.record(stream)
     stream.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     ref_check = np.isfinite(out_host.numpy()).all()
+    del graph, w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     # ---- CPU baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, heads, spent = oracle_decode_sample(cfgd, oracle_pool(cfgd), args.cpu_seconds)
+        v, heads, spent, _ = oracle_decode_sample(cfgd, oracle_pool(cfgd), args.cpu_seconds)
         threads = oracle_threads()
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": "fp64 oracle decode of %d whole KV heads (T=%d, %d query heads "
-                         "each), %.1f s of CPU work" % (heads, T, gq, spent)}
+                         "each), %.1f s of CPU work" % (heads, T, hq // hkv, spent)}
 
-    hbm, peak_kind = peaks()
+    # ---- the other workloads and the memory report (rank 0 at N = 1)
+    extra = {}
+    if rank == 0 and world == 1 and not args.no_extra and not args.seq_len:
+        pc = {}
+        for c in (1, 3, 4):
+            if c == args.config:
+                continue
+            d = dict(synth.CONFIGS[c], index=c)
+            pc[str(c)] = per_config_line(d, rank, dev, stream, hbm, 100 if c == 3 else 400)
+        extra["per_config"] = pc
+        if args.config == 2:
+            extra["memory"] = memory_report(cfgd, rank, dev, stream)
+
     value = world * step_bytes / (ms * 1e-3) / 1e9
-    achieved = per_call_bytes / (per_call_ms * 1e-3) / 1e9
+    launch_ms = ms / L  # the graph step runs only decode_kernel, L launches back to back
+    achieved = (step_bytes / L) / (launch_ms * 1e-3) / 1e9
     traffic = profile_traffic(os.path.join(ROOT, "decode_attention_13_b200", "csrc",
                                            "gtq_decode.cu"))
     n_launch = L * args.steps  # one decode_kernel launch per layer per step (graph nodes)
@@ -381,21 +563,21 @@ def run_ours(args, rank, world):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16 operands / f32 accumulate", "data": "synthetic",
-        "config": {"workload": cfgd["name"], "layers": L, "batch": B, "q_heads": hq,
-                   "kv_heads": hkv, "seq_len": T, "k_bits": kb, "v_bits": vb,
-                   "parallelism": "replicas" if world == 1 else "dp%d (independent sequences)" % world,
-                   "l2": "cold: %.0f MB of packed cache per step > 126 MB L2, layers read in turn"
-                         % (step_bytes / 1e6)},
+        "config": workload_config(cfgd, world),
         "pct_hbm_peak": 100.0 * value / world / hbm, "hbm_peak_gbs": hbm,
         "pct_hbm_nominal_8tbs": 100.0 * value / world / 8000.0,
         "ctx_tokens_per_s": world * B * T / (ms * 1e-3),
         "bytes_per_step": step_bytes,
+        "fp16_bytes_per_step": float(L * B * hkv * T * 512),
+        "compression_vs_fp16": float(L * B * hkv * T * 512) / step_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
                      "kernel": "decode_kernel: one launch per layer (query rotation, split-K "
-                               "decode and split merge fused); CUDA events around each "
-                               "layer's launch on the launching stream",
-                     "bytes_per_launch": per_call_bytes,
+                               "decode and split merge fused); average launch duration = the "
+                               "graph-timed step (CUDA events on the launching stream, only "
+                               "decode_kernel inside) divided by its %d launches" % L,
+                     "bytes_per_launch": step_bytes / L, "launch_us": 1e3 * launch_ms,
+                     "eager_call_us": 1e3 * eager_call_ms,
                      "peak_kind": peak_kind},
         "prefill": {"quantize_pack_ms_all_layers": quant_ms,
                     "quantize_pack_gbs": quant_bytes / (quant_ms * 1e-3) / 1e9,
@@ -404,6 +586,10 @@ def run_ours(args, rank, world):
                     "kernels": "quantize_tc_kernel (full 128-token tiles) + quantize_kernel "
                                "(ragged edges, none at this T); one gtq_quantize_pack call "
                                "per layer, CUDA events around all layers"},
+        "append": {"tokens_per_layer": 1, "layers": L, "ms_per_step": append_ms,
+                   "us_per_layer_token": 1e3 * append_ms / L,
+                   "how": "gtq_quantize_pack(t0 = T - 1, n = 1) on every layer, captured in a "
+                          "CUDA graph, under the allocation computed at prefill"},
         "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                 "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
@@ -414,11 +600,11 @@ def run_ours(args, rank, world):
         "clocks": clk,
         "outputs_finite": bool(ref_check),
     }
+    res.update(extra)
     if cpu:
         res["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(res), flush=True)
-    del graph
 
 
 def main():

@@ -44,7 +44,7 @@ ABI_FUNCTIONS = (
     "gtq_alloc_bits", "gtq_alloc_bits_from_energy", "gtq_quantize_pack", "gtq_decode_attn",
     "gtq_free", "gtq_packed_bytes", "gtq_get_bits", "gtq_get_energy", "gtq_status",
     "gtq_strerror", "gtq_last_error", "gtq_lloyd_max", "gtq_rotation", "gtq_layout_tile_bytes",
-    "gtq_block_energy_noalloc",
+    "gtq_block_energy_noalloc", "gtq_plan_device_bytes", "gtq_raise_status",
 )
 
 
@@ -97,6 +97,8 @@ def _load():
         "gtq_rotation": (I32, [ctypes.c_uint64, I32, I32, ctypes.POINTER(ctypes.c_double)]),
         "gtq_layout_tile_bytes": (SZ, [I32, I32]),
         "gtq_block_energy_noalloc": (I32, [ctypes.POINTER(gtq_config), P, I64, I64x4, P, P]),
+        "gtq_plan_device_bytes": (SZ, [P]),
+        "gtq_raise_status": (I32, [P, I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -239,6 +241,14 @@ def gtq_get_energy(plan: Plan, stream=None):
 
 def gtq_status(plan: Plan) -> int:
     return int(_lib.gtq_status(plan.handle))
+
+
+def gtq_plan_device_bytes(plan: Plan) -> int:
+    return int(_lib.gtq_plan_device_bytes(plan.handle))
+
+
+def gtq_raise_status(plan: Plan, code: int) -> None:
+    _check(_lib.gtq_raise_status(plan.handle, int(code)), "gtq_raise_status")
 
 
 def gtq_lloyd_max(bits: int):

@@ -224,6 +224,35 @@ int gtq_get_energy(gtq_plan* plan, double* host_energy, void* stream) {
   return cuda_code(e);
 }
 
+size_t gtq_plan_device_bytes(const gtq_plan* plan) {
+  if (!plan) return 0;
+  const size_t H = plan->n_heads;
+  size_t b = H * plan->n_blocks * sizeof(double) + H * plan->n_blocks + H * sizeof(HeadMeta) +
+             H * kD * kD * sizeof(float) + H * kRotPackBytes +
+             H * kPartialSlots * 8 * kPartialStride * sizeof(float) +
+             H * kTicketStride * sizeof(unsigned) + sizeof(int);
+  if (plan->cfg.head_dim == kD) b += H * b_image_bytes();
+  return b;
+}
+
+int gtq_raise_status(gtq_plan* plan, int32_t code) {
+  if (!plan) return GTQ_ERR_INVALID;
+  int bit = 0;
+  if (code == GTQ_ERR_TIMEOUT) bit = kStatusTimeout;
+  else if (code == GTQ_ERR_OVERFLOW) bit = kStatusOverflow;
+  else return GTQ_ERR_INVALID;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaError_t e = cudaSetDevice(plan->device);
+  int v = 0;
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, plan->d_status, sizeof(int), cudaMemcpyDeviceToHost);
+  v |= bit;
+  if (e == cudaSuccess) e = cudaMemcpy(plan->d_status, &v, sizeof(int), cudaMemcpyHostToDevice);
+  cudaSetDevice(prev);
+  return cuda_code(e);
+}
+
 int gtq_status(gtq_plan* plan) {
   if (!plan) return GTQ_ERR_INVALID;
   int v = 0;

@@ -48,7 +48,6 @@ constexpr int kMaxRing = 32;                  // stages
 constexpr int kTPS = 2;                       // tiles per stage
 constexpr int kSkip = -1;                     // stage tile slot without a tile
 constexpr int kEnd = -2;                      // no tiles left for the pair
-constexpr int kLookahead = 24;                // tiles between the L2 prefetch and the copy
 constexpr int kGrab = 2;                      // tiles per counter grab
 constexpr int kStaticEighths = 7;             // share of a head's tiles dealt out statically
 constexpr uint32_t kTabSharedAddr = 163840;   // shared address of the lookup tables
@@ -319,7 +318,10 @@ __device__ __forceinline__ void load_slot(const uint8_t* tile, int off, uint32_t
 // g + 8u for u = 4 wh .. 4 wh + 3, i.e. W bytes of each slot's 2W-byte lane
 // portion); a last run of at most 4 slots is a half k-tile (m16n8k8).  Slots
 // past the group's run within a k-tile read unrelated bits; their q is zero.
-template <int W, bool SPLIT>
+// Lookups always fetch hi and lo parts; only the groups marked split multiply
+// the lo parts (A_hi q_lo + A_lo q_hi), so one body per width serves both and
+// the hot code stays small.
+template <int W>
 __device__ __forceinline__ void group_scores(const DecodeSmem& s, const uint8_t* tile,
                                              uint4 desc, int lane_koff, const TabBase& tb,
                                              int lane, float (&C)[2][4]) {
@@ -328,53 +330,43 @@ __device__ __forceinline__ void group_scores(const DecodeSmem& s, const uint8_t*
 #pragma unroll
     for (int r = 0; r < 4; ++r) C[mt][r] = 0.f;
   const int nk16 = (desc.x >> 8) & 0xff, half = (desc.x >> 16) & 1;
-  const int kt0 = (int)desc.z;
+  const bool split = (desc.x >> 4) & 1;
+  const uint4* qf = &s.qf[desc.z][lane];
   int off = (int)desc.y + lane_koff;
 #pragma unroll 1
-  for (int k = 0; k < nk16; ++k, off += 128 * W) {
+  for (int k = 0; k < nk16; ++k, off += 128 * W, qf += 32) {
     uint32_t xa[2], xb[2];
     load_slot<W>(tile, off, xa);
     load_slot<W>(tile, off + 64 * W, xb);
-    uint4 qv;
-    if constexpr (SPLIT) {
-      qv = s.qf[kt0 + k][lane];
-    } else {
-      const uint2 hq = *reinterpret_cast<const uint2*>(&s.qf[kt0 + k][lane]);
-      qv = make_uint4(hq.x, hq.y, 0u, 0u);
-    }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      uint32_t ah[4], al[4];
-      if (mt == 0) {
-        code_pair<W, 0, SPLIT>(xa, tb, ah[0], al[0]);
-        code_pair<W, 1, SPLIT>(xa, tb, ah[1], al[1]);
-        code_pair<W, 0, SPLIT>(xb, tb, ah[2], al[2]);
-        code_pair<W, 1, SPLIT>(xb, tb, ah[3], al[3]);
-      } else {
-        code_pair<W, 2, SPLIT>(xa, tb, ah[0], al[0]);
-        code_pair<W, 3, SPLIT>(xa, tb, ah[1], al[1]);
-        code_pair<W, 2, SPLIT>(xb, tb, ah[2], al[2]);
-        code_pair<W, 3, SPLIT>(xb, tb, ah[3], al[3]);
-      }
-      mma16816(C[mt], ah, qv.x, qv.y);
-      if constexpr (SPLIT) {
-        mma16816(C[mt], ah, qv.z, qv.w);
-        mma16816(C[mt], al, qv.x, qv.y);
-      }
-    }
+    const uint4 qv = *qf;
+#define GTQ_KMT(MT)                                                  \
+  {                                                                  \
+    uint32_t ah[4], al[4];                                           \
+    code_pair<W, 2 * (MT), true>(xa, tb, ah[0], al[0]);              \
+    code_pair<W, 2 * (MT) + 1, true>(xa, tb, ah[1], al[1]);          \
+    code_pair<W, 2 * (MT), true>(xb, tb, ah[2], al[2]);              \
+    code_pair<W, 2 * (MT) + 1, true>(xb, tb, ah[3], al[3]);          \
+    mma16816(C[MT], ah, qv.x, qv.y);                                 \
+    if (split) {                                                     \
+      mma16816(C[MT], ah, qv.z, qv.w);                               \
+      mma16816(C[MT], al, qv.x, qv.y);                               \
+    }                                                                \
+  }
+    GTQ_KMT(0) GTQ_KMT(1)
+#undef GTQ_KMT
   }
   if (half) {
     uint32_t xa[2];
     load_slot<W>(tile, off, xa);
-    const uint4 qv = s.qf[kt0 + nk16][lane];
+    const uint4 qv = *qf;
     uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
-    code_pair<W, 0, SPLIT>(xa, tb, h0, l0);
-    code_pair<W, 1, SPLIT>(xa, tb, h1, l1);
-    code_pair<W, 2, SPLIT>(xa, tb, h2, l2);
-    code_pair<W, 3, SPLIT>(xa, tb, h3, l3);
+    code_pair<W, 0, true>(xa, tb, h0, l0);
+    code_pair<W, 1, true>(xa, tb, h1, l1);
+    code_pair<W, 2, true>(xa, tb, h2, l2);
+    code_pair<W, 3, true>(xa, tb, h3, l3);
     mma1688(C[0], h0, h1, qv.x);
     mma1688(C[1], h2, h3, qv.x);
-    if constexpr (SPLIT) {
+    if (split) {
       mma1688(C[0], h0, h1, qv.z);
       mma1688(C[1], h2, h3, qv.z);
       mma1688(C[0], l0, l1, qv.x);
@@ -594,9 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   if (producer) {
     // ------------------------------------------------------------ producer
     // The whole warp runs the schedule (lane 0's counter grabs are broadcast);
-    // lane 0 issues the stage copies, and every lane prefetches the cache lines
-    // of the tiles kLookahead ahead into L2 through the load path, which keeps
-    // HBM busy without holding shared memory or the copy engine.
+    // lane 0 issues the stage copies.
     {
       int fills = 0;
       if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_bar, 0))) {
@@ -611,7 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         const int64_t st0 = min((int64_t)split * a.static_per, tiles_T);
         const int64_t st1 = min(st0 + a.static_per, tiles_T);
         const int64_t dyn0 = (int64_t)nsplit * a.static_per;
-        const int64_t pf_done = st0 + a.prefetch;  // prefetched before the wait
         int64_t snext = st0;
         bool setup_ok = false, exhausted = false;
         auto grab = [&]() -> int {
@@ -635,14 +624,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             return -1;
           }
           return t;
-        };
-        const int lines = a.tile_bytes >> 7;
-        auto lookahead = [&](int64_t t) {  // static-share tiles only
-          const int64_t tp = t + kLookahead;
-          if (t < 0 || tp < pf_done || tp >= st1 || hv.pages) return;
-          const uint8_t* base = hv.tile(a.packed, tp);
-          for (int l = lane; l < lines; l += 32)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(base + ((size_t)l << 7)));
         };
         int64_t pending = next_tile();
         int ends = 0, slot = 0, round = 0;
@@ -682,8 +663,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
                                  &s.full[slot], pol);
               }
             }
-            lookahead(t0);
-            lookahead(t1);
           } else {
             // end markers: every pair meets one as its next tile slot
             if (lane == 0) {
@@ -859,13 +838,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       for (int gi = 0; gi < n_groups; ++gi) {
         const uint4 desc = s.gdesc[gi];
         float C[2][4];
-        switch (desc.x & 0x1f) {  // W | split << 4
-#define GTQ_GROUP(WW)                                                              \
-  case WW:                                                                         \
-    group_scores<WW, false>(s, tl, desc, WW * lane_kunit, tb, lane, C);            \
-    break;                                                                         \
-  case WW + 16:                                                                    \
-    group_scores<WW, true>(s, tl, desc, WW * lane_kunit, tb, lane, C);             \
+        switch (desc.x & 0xf) {  // W
+#define GTQ_GROUP(WW)                                                   \
+  case WW:                                                              \
+    group_scores<WW>(s, tl, desc, WW * lane_kunit, tb, lane, C);        \
     break;
           GTQ_GROUP(1) GTQ_GROUP(2) GTQ_GROUP(3) GTQ_GROUP(4)
           GTQ_GROUP(5) GTQ_GROUP(6) GTQ_GROUP(7) GTQ_GROUP(8)

@@ -192,6 +192,20 @@ GTQ_API int gtq_get_energy(gtq_plan* plan, double* host_energy, void* stream);
  * plan's split-merge state: free the plan and build a new one. */
 GTQ_API int gtq_status(gtq_plan* plan);
 
+/* Device memory owned by the plan, in bytes (0 on NULL): energies, widths,
+ * metadata, rotation rows and images, split-merge partials and counters; the
+ * per-device constant tables and the caller's buffers are not counted. */
+GTQ_API size_t gtq_plan_device_bytes(const gtq_plan* plan);
+
+/*
+ * gtq_raise_status -- set a condition in the plan's device status word from
+ * the host, exactly as a kernel does when it meets it (code GTQ_ERR_TIMEOUT:
+ * a bounded wait expired; GTQ_ERR_OVERFLOW: a norm was clamped).  It lets a
+ * caller test its handling of gtq_status without making a GPU fault or hang.
+ * Synchronises the device.  Errors: INVALID (NULL plan or another code), CUDA.
+ */
+GTQ_API int gtq_raise_status(gtq_plan* plan, int32_t code);
+
 /* Human-readable name of a return code (static string). */
 GTQ_API const char* gtq_strerror(int code);
 

@@ -126,3 +126,9 @@ def test_noalloc_energy_rejects_head_count_overflow():
         rc = lib.gtq_block_energy_noalloc(ctypes.byref(cfg), 0x1000, 64, st, 0x1000, None)
         assert rc == gtq.GTQ_ERR_INVALID
         assert "65535" in lib.gtq_last_error().decode()
+
+
+def test_status_helpers_reject_null_plan():
+    lib = gtq.binding._lib
+    assert lib.gtq_raise_status(None, gtq.GTQ_ERR_TIMEOUT) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_plan_device_bytes(None) == 0

@@ -305,3 +305,33 @@ def test_config0_as_stated():
     # the quantized decode stays close to unquantized attention on this head
     exact = attention.attention_exact(hd["q"], hd["k"], hd["v"])
     assert rel_l2(ref[0], exact) < 0.25
+
+
+@pytest.mark.parametrize("pairing,dtype", [(0, "fp16"), (1, "fp16"), (0, "fp32")])
+def test_append_under_frozen_allocation(pairing, dtype):
+    # the serving loop: widths are chosen from a prefix of T_p tokens, the
+    # prefix is quantized, then tokens are appended one or a few at a time with
+    # those widths, and the decode covers every token written so far
+    T_p, extra = 640, 16
+    c = Case(1, 2, 4, T_p + extra, 3, 3, pairing=pairing, dtype=dtype, seed=61)
+    c.plan = gtq.gtq_alloc_bits(c.cfg, c.k, T_p)            # energies of the prefix only
+    gtq.gtq_quantize_pack(c.plan, c.k, c.v, 0, T_p, c.packed)
+    bits_gpu = gtq.gtq_get_bits(c.plan)
+    t = T_p
+    for n in (1, 1, 2, 4, 8):                                 # 16 appended tokens
+        gtq.gtq_quantize_pack(c.plan, c.k, c.v, t, n, c.packed)
+        t += n
+        c.T = t
+        out = c.decode()                                      # same stream, no sync between
+        ref = np.zeros_like(out, dtype=np.float64)
+        for h in range(c.hkv):
+            k = c.lay["k"][0, h]
+            bits = allocation.greedy_bits(allocation.block_energy(k[:T_p], pairing), 3, 128)
+            assert np.array_equal(bits_gpu[0, h].astype(np.int64), bits)
+            kg = quantize.quantize_keys(k[:t], bits, pairing)   # all tokens, prefix widths
+            vg = quantize.quantize_values(c.lay["v"][0, h][:t], 3)
+            compare_codes(c, 0, h, kg, vg, bits)
+            q = c.lay["q"][0, h * c.gq:(h + 1) * c.gq]
+            ref[0, h * c.gq:(h + 1) * c.gq] = attention.decode_rotated(q, kg, vg)
+        assert rel_l2(out, ref) <= DECODE_REL_L2, t
+    assert gtq.gtq_status(c.plan) == gtq.GTQ_OK
