@@ -25,6 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgtq.so")
 
 GTQ_OK = 0
+GTQ_T0_TAIL = -1  # gtq_quantize_pack_ex: write the last n tokens of every sequence
 GTQ_ERR_INVALID = -1
 GTQ_ERR_UNSUPPORTED = -2
 GTQ_ERR_CUDA = -3
@@ -45,6 +46,7 @@ ABI_FUNCTIONS = (
     "gtq_free", "gtq_packed_bytes", "gtq_get_bits", "gtq_get_energy", "gtq_status",
     "gtq_strerror", "gtq_last_error", "gtq_lloyd_max", "gtq_rotation", "gtq_layout_tile_bytes",
     "gtq_block_energy_noalloc", "gtq_plan_device_bytes", "gtq_raise_status",
+    "gtq_alloc_bits_ex", "gtq_quantize_pack_ex", "gtq_decode_attn_ex",
 )
 
 
@@ -66,6 +68,26 @@ class gtq_config(ctypes.Structure):
         ("in_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
         ("seed", ctypes.c_uint64), ("t_capacity", ctypes.c_int64),
     ]
+
+
+class gtq_seq_layout(ctypes.Structure):
+    _fields_ = [
+        ("seq_lens_dev", ctypes.c_void_p), ("block_table_dev", ctypes.c_void_p),
+        ("max_blocks", ctypes.c_int64),
+    ]
+
+
+def seq_layout(seq_lens=None, block_table=None):
+    """A gtq_seq_layout from device int32 tensors: lengths [batch] and a block
+    table [batch][max_blocks] (either may be None).  Keep the tensors alive
+    while the calls that use the layout run."""
+    lay = gtq_seq_layout(None, None, 0)
+    if seq_lens is not None:
+        lay.seq_lens_dev = _ptr(seq_lens)
+    if block_table is not None:
+        lay.block_table_dev = _ptr(block_table)
+        lay.max_blocks = int(block_table.shape[1])
+    return lay
 
 
 def make_config(batch, n_q_heads, n_kv_heads, k_bits, v_bits, t_capacity, head_dim=128,
@@ -99,6 +121,11 @@ def _load():
         "gtq_block_energy_noalloc": (I32, [ctypes.POINTER(gtq_config), P, I64, I64x4, P, P]),
         "gtq_plan_device_bytes": (SZ, [P]),
         "gtq_raise_status": (I32, [P, I32]),
+        "gtq_alloc_bits_ex": (I32, [ctypes.POINTER(gtq_config), P, I64, I64x4,
+                                    ctypes.POINTER(gtq_seq_layout), P, ctypes.POINTER(P)]),
+        "gtq_quantize_pack_ex": (I32, [P, P, P, I64x4, I64, I64, P, SZ,
+                                       ctypes.POINTER(gtq_seq_layout), P]),
+        "gtq_decode_attn_ex": (I32, [P, P, I64, ctypes.POINTER(gtq_seq_layout), P, I32, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -209,6 +236,40 @@ def gtq_decode_attn(plan: Plan, packed, T: int, q, out, stream=None, q_dtype=Non
     rc = _lib.gtq_decode_attn(plan.handle, _ptr(packed), int(T), _ptr(q), int(q_dtype),
                               _ptr(out), _stream(stream))
     _check(rc, "gtq_decode_attn")
+
+
+def _lay(layout):
+    return None if layout is None else ctypes.byref(layout)
+
+
+def gtq_alloc_bits_ex(cfg: gtq_config, k, T: int, layout=None, stream=None,
+                      strides=None) -> Plan:
+    out = ctypes.c_void_p()
+    rc = _lib.gtq_alloc_bits_ex(ctypes.byref(cfg), _ptr(k), int(T), _strides4(k, strides),
+                                _lay(layout), _stream(stream), ctypes.byref(out))
+    _check(rc, "gtq_alloc_bits_ex")
+    return Plan(out.value, cfg)
+
+
+def gtq_quantize_pack_ex(plan: Plan, k, v, t0: int, n_tokens: int, packed, layout=None,
+                         stream=None, strides=None, packed_bytes=None) -> None:
+    nbytes = packed_bytes if packed_bytes is not None else (
+        packed.numel() * packed.element_size())
+    rc = _lib.gtq_quantize_pack_ex(plan.handle, _ptr(k), _ptr(v), _strides4(k, strides),
+                                   int(t0), int(n_tokens), _ptr(packed), int(nbytes),
+                                   _lay(layout), _stream(stream))
+    _check(rc, "gtq_quantize_pack_ex")
+
+
+def gtq_decode_attn_ex(plan: Plan, packed, T: int, q, out, layout=None, stream=None,
+                       q_dtype=None) -> None:
+    if q_dtype is None:
+        import torch
+
+        q_dtype = DTYPE_FP32 if q.dtype == torch.float32 else DTYPE_FP16
+    rc = _lib.gtq_decode_attn_ex(plan.handle, _ptr(packed), int(T), _lay(layout), _ptr(q),
+                                 int(q_dtype), _ptr(out), _stream(stream))
+    _check(rc, "gtq_decode_attn_ex")
 
 
 def gtq_free(plan: Plan) -> None:

@@ -46,11 +46,13 @@ template <typename T>
 __global__ void __launch_bounds__(256) energy_partial_kernel(const T* __restrict__ k, int64_t s0,
                                                              int64_t s1, int64_t s2, int hkv,
                                                              int d, int64_t T_tok,
+                                                             const int32_t* __restrict__ seq_lens,
                                                              double* __restrict__ part) {
   const int head = blockIdx.y, b = head / hkv, h = head % hkv;
   const int tl = threadIdx.x >> 4, dl = threadIdx.x & 15;
+  const int64_t T_b = seq_lens ? max((int64_t)0, min((int64_t)seq_lens[b], T_tok)) : T_tok;
   const int64_t t_begin = (int64_t)blockIdx.x * kEnergyChunk;
-  const int64_t t_end = min(t_begin + kEnergyChunk, T_tok);
+  const int64_t t_end = min(t_begin + kEnergyChunk, T_b);
   double acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0;
@@ -77,9 +79,12 @@ __global__ void __launch_bounds__(256) energy_partial_kernel(const T* __restrict
 
 // grid heads, 64 threads (one per block)
 __global__ void energy_finish_kernel(const double* __restrict__ part, int chunks, int d,
-                                     int pairing, int64_t T_tok, double* __restrict__ energy) {
+                                     int pairing, int64_t T_tok, const int32_t* __restrict__ seq_lens,
+                                     int hkv, double* __restrict__ energy) {
   const int head = blockIdx.x, i = threadIdx.x, nb = d / 2;
   if (i >= nb) return;
+  const int64_t T_b =
+      seq_lens ? max((int64_t)0, min((int64_t)seq_lens[head / hkv], T_tok)) : T_tok;
   const int p0 = pairing == GTQ_PAIRING_HALF ? i : 2 * i;
   const int p1 = pairing == GTQ_PAIRING_HALF ? i + nb : 2 * i + 1;
   double s0 = 0.0, s1 = 0.0;
@@ -87,7 +92,7 @@ __global__ void energy_finish_kernel(const double* __restrict__ part, int chunks
     s0 += part[((size_t)head * chunks + c) * 128 + p0];
     s1 += part[((size_t)head * chunks + c) * 128 + p1];
   }
-  energy[(size_t)head * nb + i] = (s0 + s1) / (double)T_tok;
+  energy[(size_t)head * nb + i] = T_b > 0 ? (s0 + s1) / (double)T_b : 0.0;
 }
 
 // one warp per head
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(128) meta_kernel(const uint8_t* __restrict__ b
 }  // namespace
 
 cudaError_t launch_energy(const gtq_plan* p, const void* k, int64_t T, const int64_t* st,
-                          cudaStream_t s) {
+                          const int32_t* seq_lens, cudaStream_t s) {
   const int chunks = (int)((T + kEnergyChunk - 1) / kEnergyChunk);
   double* part = nullptr;
   cudaError_t e = cudaMallocAsync((void**)&part, (size_t)p->n_heads * chunks * 128 * sizeof(double), s);
@@ -256,12 +261,12 @@ cudaError_t launch_energy(const gtq_plan* p, const void* k, int64_t T, const int
   const int d = p->cfg.head_dim;
   if (p->cfg.in_dtype == GTQ_DTYPE_FP16)
     energy_partial_kernel<__half><<<grid, 256, 0, s>>>((const __half*)k, st[0], st[1], st[2],
-                                                       p->cfg.n_kv_heads, d, T, part);
+                                                       p->cfg.n_kv_heads, d, T, seq_lens, part);
   else
     energy_partial_kernel<float><<<grid, 256, 0, s>>>((const float*)k, st[0], st[1], st[2],
-                                                      p->cfg.n_kv_heads, d, T, part);
+                                                      p->cfg.n_kv_heads, d, T, seq_lens, part);
   energy_finish_kernel<<<p->n_heads, 64, 0, s>>>(part, chunks, d, p->cfg.rope_pairing, T,
-                                                 p->d_energy);
+                                                 seq_lens, p->cfg.n_kv_heads, p->d_energy);
   e = cudaGetLastError();
   cudaFreeAsync(part, s);
   return e;
@@ -372,12 +377,14 @@ extern "C" int gtq_block_energy_noalloc(const gtq_config* cfg, const void* k_dev
   if (cfg->in_dtype == GTQ_DTYPE_FP16)
     energy_partial_kernel<__half><<<grid, 256, 0, s>>>((const __half*)k_dev, k_strides[0],
                                                        k_strides[1], k_strides[2],
-                                                       cfg->n_kv_heads, cfg->head_dim, T, part);
+                                                       cfg->n_kv_heads, cfg->head_dim, T, nullptr,
+                                                       part);
   else
     energy_partial_kernel<float><<<grid, 256, 0, s>>>((const float*)k_dev, k_strides[0],
                                                       k_strides[1], k_strides[2],
-                                                      cfg->n_kv_heads, cfg->head_dim, T, part);
+                                                      cfg->n_kv_heads, cfg->head_dim, T, nullptr,
+                                                      part);
   energy_finish_kernel<<<heads, 64, 0, s>>>(part, (int)chunks, cfg->head_dim, cfg->rope_pairing,
-                                            T, energy_dev);
+                                            T, nullptr, cfg->n_kv_heads, energy_dev);
   return record_cuda_error(cudaGetLastError());
 }

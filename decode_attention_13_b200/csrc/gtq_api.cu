@@ -105,9 +105,32 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   return GTQ_OK;
 }
 
+// a layout's pointers and sizes (its contents live on the device)
+int check_layout(const gtq_seq_layout* lay, int64_t T) {
+  if (!lay) return GTQ_OK;
+  if (lay->seq_lens_dev && !aligned(lay->seq_lens_dev, 4)) return GTQ_ERR_INVALID;
+  if (lay->block_table_dev) {
+    if (!aligned(lay->block_table_dev, 4) || lay->max_blocks < 1) return GTQ_ERR_INVALID;
+    if ((T + kTile - 1) / kTile > lay->max_blocks) return GTQ_ERR_INVALID;
+  }
+  return GTQ_OK;
+}
+
 }  // namespace
 
 namespace gtq {
+SeqMap seq_map(const gtq_plan* p, const gtq_seq_layout* lay) {
+  SeqMap m;
+  m.hkv = p->cfg.n_kv_heads;
+  m.n_tiles = p->n_tiles;
+  m.tile_bytes = (int64_t)p->tile_bytes;
+  if (lay) {
+    m.seq_lens = lay->seq_lens_dev;
+    m.table = lay->block_table_dev;
+    m.max_blocks = lay->block_table_dev ? lay->max_blocks : 0;
+  }
+  return m;
+}
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 int record_cuda_error(cudaError_t e) { return cuda_code(e); }
 }  // namespace gtq
@@ -121,7 +144,14 @@ size_t gtq_layout_tile_bytes(int32_t k_bits, int32_t v_bits) {
 
 int gtq_alloc_bits(const gtq_config* cfg, const void* k_dev, int64_t T, const int64_t k_strides[4],
                    void* stream, gtq_plan** out) {
+  return gtq_alloc_bits_ex(cfg, k_dev, T, k_strides, nullptr, stream, out);
+}
+
+int gtq_alloc_bits_ex(const gtq_config* cfg, const void* k_dev, int64_t T,
+                      const int64_t k_strides[4], const gtq_seq_layout* lay, void* stream,
+                      gtq_plan** out) {
   if (!out || !k_dev || !k_strides) return GTQ_ERR_INVALID;
+  if (lay && lay->seq_lens_dev && !aligned(lay->seq_lens_dev, 4)) return GTQ_ERR_INVALID;
   int rc = check_config(cfg, false);
   if (rc != GTQ_OK) return rc;
   if (cfg->head_dim % 8) return GTQ_ERR_UNSUPPORTED;  // energy pass reads 8-dim vectors
@@ -134,7 +164,7 @@ int gtq_alloc_bits(const gtq_config* cfg, const void* k_dev, int64_t T, const in
   rc = make_plan(cfg, &p);
   if (rc != GTQ_OK) return rc;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_energy(p, k_dev, T, k_strides, s);
+  cudaError_t e = launch_energy(p, k_dev, T, k_strides, lay ? lay->seq_lens_dev : nullptr, s);
   if (e == cudaSuccess) e = launch_greedy_and_meta(p, s);
   if (e != cudaSuccess) {
     cudaStreamSynchronize(s);
@@ -168,28 +198,51 @@ int gtq_alloc_bits_from_energy(const gtq_config* cfg, const double* host_energy,
 int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_dev,
                       const int64_t strides[4], int64_t t0, int64_t n_tokens, void* packed_dev,
                       size_t packed_bytes, void* stream) {
+  return gtq_quantize_pack_ex(plan, k_dev, v_dev, strides, t0, n_tokens, packed_dev, packed_bytes,
+                              nullptr, stream);
+}
+
+int gtq_quantize_pack_ex(gtq_plan* plan, const void* k_dev, const void* v_dev,
+                         const int64_t strides[4], int64_t t0, int64_t n_tokens, void* packed_dev,
+                         size_t packed_bytes, const gtq_seq_layout* lay, void* stream) {
   if (!plan || !k_dev || !v_dev || !strides || !packed_dev) return GTQ_ERR_INVALID;
   if (plan->cfg.head_dim != kD) return GTQ_ERR_UNSUPPORTED;
+  const bool tail = t0 == GTQ_T0_TAIL;
+  if (tail && !(lay && lay->seq_lens_dev)) return GTQ_ERR_INVALID;
+  if (tail) t0 = 0;  // the range checks below then bound n_tokens by the capacity
   if (t0 < 0 || n_tokens < 1 || t0 + n_tokens > plan->cfg.t_capacity) return GTQ_ERR_INVALID;
-  if (packed_bytes < plan->packed_bytes || !aligned(packed_dev, 16)) return GTQ_ERR_INVALID;
+  const bool paged = lay && lay->block_table_dev;
+  const size_t need = paged ? (size_t)plan->cfg.n_kv_heads * plan->tile_bytes : plan->packed_bytes;
+  if (packed_bytes < need || !aligned(packed_dev, 16)) return GTQ_ERR_INVALID;
+  if (check_layout(lay, tail ? plan->cfg.t_capacity : t0 + n_tokens) != GTQ_OK)
+    return GTQ_ERR_INVALID;
   const int esz = plan->cfg.in_dtype == GTQ_DTYPE_FP16 ? 2 : 4;
   if (strides[3] != 1 || !aligned(k_dev, esz) || !aligned(v_dev, esz)) return GTQ_ERR_INVALID;
   for (int i = 0; i < 3; ++i)
     if (strides[i] < 0) return GTQ_ERR_INVALID;
+  SeqMap sm = seq_map(plan, lay);
+  sm.tail = tail ? 1 : 0;
   return cuda_code(launch_quantize(plan, k_dev, v_dev, strides, t0, n_tokens,
-                                   (uint8_t*)packed_dev, (cudaStream_t)stream));
+                                   (uint8_t*)packed_dev, sm, (cudaStream_t)stream));
 }
 
 int gtq_decode_attn(gtq_plan* plan, const void* packed_dev, int64_t T, const void* q_dev,
                     int32_t q_dtype, float* out_dev, void* stream) {
+  return gtq_decode_attn_ex(plan, packed_dev, T, nullptr, q_dev, q_dtype, out_dev, stream);
+}
+
+int gtq_decode_attn_ex(gtq_plan* plan, const void* packed_dev, int64_t T,
+                       const gtq_seq_layout* lay, const void* q_dev, int32_t q_dtype,
+                       float* out_dev, void* stream) {
   if (!plan || !packed_dev || !q_dev || !out_dev) return GTQ_ERR_INVALID;
   if (plan->cfg.head_dim != kD) return GTQ_ERR_UNSUPPORTED;
   if (T < 1 || T > plan->cfg.t_capacity) return GTQ_ERR_INVALID;
   if (q_dtype != GTQ_DTYPE_FP16 && q_dtype != GTQ_DTYPE_FP32) return GTQ_ERR_INVALID;
   if (!aligned(packed_dev, 16) || !aligned(q_dev, 16) || !aligned(out_dev, 16))
     return GTQ_ERR_INVALID;
+  if (check_layout(lay, T) != GTQ_OK) return GTQ_ERR_INVALID;
   return cuda_code(launch_decode(plan, (const uint8_t*)packed_dev, T, q_dev, q_dtype, out_dev,
-                                 (cudaStream_t)stream));
+                                 seq_map(plan, lay), (cudaStream_t)stream));
 }
 
 int gtq_free(gtq_plan* plan) {

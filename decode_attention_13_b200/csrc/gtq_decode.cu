@@ -1108,7 +1108,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }  // namespace
 
 cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, const void* q,
-                          int q_dtype, float* out, cudaStream_t s) {
+                          int q_dtype, float* out, const SeqMap& sm, cudaStream_t s) {
   DecodeArgs a;
   a.packed = packed;
   a.meta = p->d_meta;
@@ -1123,9 +1123,9 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.dec_image = p->tab.dec_image;
   a.partials = p->d_partials;
   a.status = p->d_status;
-  a.seq_lens = nullptr;
-  a.block_table = nullptr;
-  a.max_blocks = 0;
+  a.seq_lens = sm.seq_lens;
+  a.block_table = sm.table;
+  a.max_blocks = sm.max_blocks;
   a.T = T;
   a.n_tiles = p->n_tiles;
   a.tile_bytes = (int)p->tile_bytes;

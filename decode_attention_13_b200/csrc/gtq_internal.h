@@ -128,10 +128,38 @@ static_assert(sizeof(CodeLutMeta) <= kCodeLutHeader - 4, "code LUT header");
 constexpr int kCodeLutOkOffset = kCodeLutHeader - 4;  // int: 1 when the table is valid
 constexpr size_t kCodeLutBytes = kCodeLutHeader + kCodeLutEntries * 8;
 
+// Where the packed tile t of head (b, h) lives and how many tokens sequence b
+// holds: contiguous per head (tile t of head at (head * n_tiles + t) tiles), or
+// paged (block table row b: page table[b][t] holds tile t of every KV head of
+// sequence b, head h at (page * hkv + h) tiles); lengths from seq_lens[b]
+// (clamped to T) or T for all.
+struct SeqMap {
+  const int32_t* seq_lens = nullptr;
+  const int32_t* table = nullptr;
+  int64_t max_blocks = 0;
+  int tail = 0;  // quantize: write the last n tokens of each sequence (t0 ignored)
+  int hkv = 1;
+  int64_t n_tiles = 0;
+  int64_t tile_bytes = 0;
+  __device__ __forceinline__ int64_t len(int b, int64_t T) const {
+    if (!seq_lens) return T;
+    const int64_t l = seq_lens[b];
+    return l < 0 ? 0 : (l < T ? l : T);
+  }
+  __device__ __forceinline__ uint8_t* tile(uint8_t* packed, int head, int64_t t) const {
+    if (table) {
+      const int b = head / hkv, h = head % hkv;
+      return packed + ((int64_t)table[(int64_t)b * max_blocks + t] * hkv + h) * tile_bytes;
+    }
+    return packed + ((int64_t)head * n_tiles + t) * tile_bytes;
+  }
+};
+
 // Device-resident constant tables shared by every plan of a (device, seed).
 struct Tables {
   double* rot_k;     // R_m for m = 2, 4, ..., 128, row-major, concatenated (fp64)
   float* rot_v;      // R_V 128 x 128 row-major (fp32)
+  float* rot_vt;     // R_V^T (fp32): element [d][r] = R_V[r][d]
   double* dist;      // D(0..8)
   float* thr;        // fp32 thresholds, width w at thr_base(w)
   uint4* dec_image;  // kDecodeImageBytes: the decode kernel's lookup tables
@@ -183,18 +211,25 @@ int tables_for(int device, uint64_t seed, Tables* out);  // cached per (device, 
 
 // Kernel launchers
 cudaError_t launch_energy(const gtq_plan* p, const void* k, int64_t T, const int64_t* st,
-                          cudaStream_t s);
+                          const int32_t* seq_lens, cudaStream_t s);
+SeqMap seq_map(const gtq_plan* p, const gtq_seq_layout* lay);
 cudaError_t launch_greedy_and_meta(const gtq_plan* p, cudaStream_t s);
 cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                            int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s);
+                            int64_t t0, int64_t n, uint8_t* packed, const SeqMap& sm,
+                            cudaStream_t s);
 cudaError_t launch_quantize_cc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                               int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s);
+                               int64_t t0, int64_t n, uint8_t* packed, const SeqMap& sm,
+                               cudaStream_t s);
+constexpr int kAppendMax = 16;  // tokens per call handled by the append kernel
+cudaError_t launch_append(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                          int64_t t0, int64_t n, uint8_t* packed, const SeqMap& sm, cudaStream_t s);
 cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                               int64_t mt0, int64_t mt1, uint8_t* packed, cudaStream_t s);
+                               int64_t mt0, int64_t mt1, uint8_t* packed, const SeqMap& sm,
+                               cudaStream_t s);
 cudaError_t build_b_images(const float* rows, int count, size_t stride, uint8_t* img,
                            cudaStream_t s);
 size_t b_image_bytes();
 cudaError_t build_code_lut(const float* thr, uint8_t* blob, cudaStream_t s);
 cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, const void* q,
-                          int q_dtype, float* out, cudaStream_t s);
+                          int q_dtype, float* out, const SeqMap& sm, cudaStream_t s);
 }  // namespace gtq

@@ -38,6 +38,8 @@ struct QuantArgs {
   int tile_bytes;
   int kb, vb;
   int* status;
+  SeqMap sm;       // tile addresses and sequence lengths
+  int64_t cap;     // t_capacity: lengths are clamped to it
 };
 
 struct QuantSmem {
@@ -126,6 +128,11 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
   uint32_t* img32 = reinterpret_cast<uint32_t*>(img);
   const int head = blockIdx.y, b = head / a.hkv, h = head % a.hkv;
   const int tid = threadIdx.x;
+  // this sequence's tokens of the call: [t0, t1)
+  const int64_t len = a.sm.len(b, a.cap);
+  const int64_t t0 = a.sm.tail ? max((int64_t)0, len - a.n) : a.t0;
+  const int64_t t1 = a.sm.tail ? len : min(a.t0 + a.n, len);
+  if (t1 <= t0) return;
 
   if (tid == 0) {
     s.meta = a.meta[head];
@@ -144,19 +151,19 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
   const T* vbase = reinterpret_cast<const T*>(a.v) + b * a.s0 + h * a.s1;
   const int vcode_off = 1024 * a.kb, vnorm_off = 1024 * (a.kb + a.vb);
   const int knorm_off = vnorm_off + 128;
-  const int64_t tile_first = a.t0 / kTile, tile_last = (a.t0 + a.n - 1) / kTile;
+  const int64_t tile_first = t0 / kTile, tile_last = (t1 - 1) / kTile;
   const int tb = tid >> 4, rb = tid & 15;
   const float sqrt_d = sqrtf((float)kD);
 
   for (int64_t tile = tile_first + blockIdx.x; tile <= tile_last; tile += gridDim.x) {
     const int64_t tok0 = tile * kTile;
-    const bool full = tok0 >= a.t0 && tok0 + kTile <= a.t0 + a.n;
-    uint8_t* gimg = a.packed + ((size_t)head * a.n_tiles + tile) * a.tile_bytes;
+    const bool full = tok0 >= t0 && tok0 + kTile <= t1;
+    uint8_t* gimg = a.sm.tile(a.packed, head, tile);
     for (int i = tid; i < a.tile_bytes / 16; i += kQThreads)
       reinterpret_cast<uint4*>(img)[i] =
           full ? make_uint4(0, 0, 0, 0) : reinterpret_cast<const uint4*>(gimg)[i];
     // ------------------------------------------------------------------- keys
-    load_tile<T>(s, kbase, tok0, a.t0, a.n, a.s2);
+    load_tile<T>(s, kbase, tok0, t0, t1 - t0, a.s2);
     __syncthreads();
     for (int task = tid; task < kTile * m.n_groups; task += kQThreads) {
       const int j = task % kTile, g = task / kTile;
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
       }
       const double nrm = sqrt(acc);
       s.scale[j][g] = nrm > 0.0 ? (float)((double)m.sqrt_m[g] / nrm) : 0.f;
-      if (t >= a.t0 && t < a.t0 + a.n) {
+      if (t >= t0 && t < t1) {
         int ovf = 0;
         const __half hn = norm_to_half(nrm, &ovf);
         if (ovf) s.overflow = 1;
@@ -208,14 +215,14 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
         for (int u = 0; u < 8; ++u) {
           const int j = g + 8 * u;
           const int64_t t = tok0 + j;
-          if (t < a.t0 || t >= a.t0 + a.n) continue;
+          if (t < t0 || t >= t1) continue;
           for (int e = 0; e < 2; ++e)
             put_bits(base, g * 16 * w + (2 * u + e) * w, s.codes[j][2 * slot + e], w);
         }
     }
     __syncthreads();
     // ----------------------------------------------------------------- values
-    load_tile<T>(s, vbase, tok0, a.t0, a.n, a.s2);
+    load_tile<T>(s, vbase, tok0, t0, t1 - t0, a.s2);
     __syncthreads();
     if (tid < kTile) {
       const int j = tid;
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
       }
       const double nrm = sqrt(acc);
       s.scale[j][0] = nrm > 0.0 ? (float)((double)sqrt_d / nrm) : 0.f;
-      if (t >= a.t0 && t < a.t0 + a.n) {
+      if (t >= t0 && t < t1) {
         int ovf = 0;
         const __half hn = norm_to_half(nrm, &ovf);
         if (ovf) s.overflow = 1;
@@ -256,7 +263,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
         const int dim = 16 * i + g + 8 * ((x >> 1) & 1);
         const int j = 16 * (x >> 3) + 2 * c + (x & 1) + 8 * ((x >> 2) & 1);
         const int64_t t = tok0 + j;
-        if (t < a.t0 || t >= a.t0 + a.n) continue;
+        if (t < t0 || t >= t1) continue;
         put_bits(base, x * a.vb, s.codes[j][dim], a.vb);
       }
     }
@@ -271,7 +278,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
 }  // namespace
 
 cudaError_t launch_quantize_cc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                               int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s) {
+                               int64_t t0, int64_t n, uint8_t* packed, const SeqMap& sm,
+                               cudaStream_t s) {
   QuantArgs a;
   a.k = k; a.v = v;
   a.s0 = st[0]; a.s1 = st[1]; a.s2 = st[2];
@@ -288,8 +296,10 @@ cudaError_t launch_quantize_cc(const gtq_plan* p, const void* k, const void* v, 
   a.kb = p->cfg.k_bits;
   a.vb = p->cfg.v_bits;
   a.status = p->d_status;
+  a.sm = sm;
+  a.cap = p->cfg.t_capacity;
   const size_t smem = kImgOffset + p->tile_bytes;
-  const int64_t tiles = (t0 + n - 1) / kTile - t0 / kTile + 1;
+  const int64_t tiles = sm.tail ? (n + kTile - 1) / kTile + 1 : (t0 + n - 1) / kTile - t0 / kTile + 1;
   int per_head = (int)std::min<int64_t>(tiles, std::max(1, (p->n_sms + p->n_heads - 1) / p->n_heads));
   dim3 grid(per_head, p->n_heads);
   cudaError_t e;
@@ -309,22 +319,33 @@ cudaError_t launch_quantize_cc(const gtq_plan* p, const void* k, const void* v, 
 
 // Whole 128-token tiles of fp16 inputs go to the tensor-core kernel; the ragged
 // edges (partial packed tiles, appends) and fp32 inputs to the CUDA-core kernel.
+// Tokens [t0, t0 + n) outside the tensor-core tiles: a few tokens (a
+// decode-time append) go to the append kernel, more to the CUDA-core kernel.
+static cudaError_t launch_edge(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
+                               int64_t t0, int64_t n, uint8_t* packed, const SeqMap& sm,
+                               cudaStream_t s) {
+  if (n <= kAppendMax) return launch_append(p, k, v, st, t0, n, packed, sm, s);
+  return launch_quantize_cc(p, k, v, st, t0, n, packed, sm, s);
+}
+
 cudaError_t launch_quantize(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                            int64_t t0, int64_t n, uint8_t* packed, cudaStream_t s) {
+                            int64_t t0, int64_t n, uint8_t* packed, const SeqMap& sm,
+                            cudaStream_t s) {
+  if (sm.tail) return launch_edge(p, k, v, st, 0, n, packed, sm, s);  // starts per sequence
   if (p->cfg.in_dtype == GTQ_DTYPE_FP16 && p->cfg.head_dim == kD) {
     const int64_t mt0 = (t0 + 127) / 128, mt1 = (t0 + n) / 128;
     if (mt1 > mt0) {
-      cudaError_t e = launch_quantize_tc(p, k, v, st, mt0, mt1, packed, s);
+      cudaError_t e = launch_quantize_tc(p, k, v, st, mt0, mt1, packed, sm, s);
       if (e != cudaErrorNotSupported) {
         if (e != cudaSuccess) return e;
-        if (mt0 * 128 > t0) e = launch_quantize_cc(p, k, v, st, t0, mt0 * 128 - t0, packed, s);
+        if (mt0 * 128 > t0) e = launch_edge(p, k, v, st, t0, mt0 * 128 - t0, packed, sm, s);
         if (e == cudaSuccess && t0 + n > mt1 * 128)
-          e = launch_quantize_cc(p, k, v, st, mt1 * 128, t0 + n - mt1 * 128, packed, s);
+          e = launch_edge(p, k, v, st, mt1 * 128, t0 + n - mt1 * 128, packed, sm, s);
         return e;
       }
     }
   }
-  return launch_quantize_cc(p, k, v, st, t0, n, packed, s);
+  return launch_edge(p, k, v, st, t0, n, packed, sm, s);
 }
 
 }  // namespace gtq

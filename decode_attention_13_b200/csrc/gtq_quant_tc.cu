@@ -115,6 +115,8 @@ struct TcArgs {
   int64_t mt0, mt1;       // MMA tiles [mt0, mt1) of every head
   int ctas_k, ctas_v;     // CTAs per head of each role (blockIdx.x < ctas_k: keys)
   int* status;
+  SeqMap sm;              // tile addresses and sequence lengths
+  int64_t cap;            // t_capacity: lengths are clamped to it
 };
 
 __device__ __forceinline__ uint32_t su32(const void* p) {
@@ -331,6 +333,8 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
   uint8_t* sm = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = su32(sm);
   const int head = blockIdx.y, bidx = head / a.hkv, hidx = head % a.hkv;
+  // tokens of this sequence: packed tiles starting at or past len are not written
+  const int64_t len = a.sm.len(bidx, a.cap);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* scale = reinterpret_cast<float*>(sm + kOffScale);
   uint8_t* zflags = sm + kOffFlags;
@@ -491,8 +495,9 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       }
       if (!mbar_wait(bar(kSEmpty + par), ((it >> 1) & 1) ^ 1)) { failed = 1; break; }
       tc_fence_after();
-      uint8_t* tile_base =
-          a.packed + ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + (j >> 6))) * a.tile_bytes;
+      const int64_t tok = (a.mt0 + t) * 128 + j;
+      const bool tile_ok = (tok & ~int64_t(63)) < len, tok_ok = tok < len;
+      uint8_t* tile_base = tile_ok ? a.sm.tile(a.packed, head, (a.mt0 + t) * 2 + (j >> 6)) : nullptr;
       const uint8_t* xt = sm + kOffA + st * kStageBytes;
       float* sc_par = scale + par * kMaxGroups * kScaleStride;
       // Group sums of exact squares in fp32 (eight accumulators), and each group's
@@ -519,14 +524,15 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
         const uint16_t l16 = __half_as_ushort(__float2half_rn(fminf(lo, 65504.f)));
         const uint16_t h16 = __half_as_ushort(__float2half_rn(fminf(hi, 65504.f)));
         zm |= zero ? 1u : 0u;
-        ovf |= over ? 1 : 0;
+        ovf |= (over && tok_ok) ? 1 : 0;
         ambm |= ((zero || over) ? 0u : (strad ? 2u : (l16 != h16 ? 1u : 0u))) << (2 * g);
         const uint32_t pk = (uint32_t)l16 | ((uint32_t)h16 << 16);
 #pragma unroll
         for (int gg = 0; gg < kMaxGroups; ++gg)
           if (gg == g) lh[gg] = pk;
-        *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) =
-            zero ? (uint16_t)0 : (over ? (uint16_t)0x7BFF : l16);
+        if (tile_ok)
+          *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) =
+              zero ? (uint16_t)0 : (over ? (uint16_t)0x7BFF : l16);
         // scale of the codes (fp32, about 2^-22 relative)
         sc_par[g * kScaleStride + j] = zero ? 0.f : gi.sqrt_m[g] * r;
       };
@@ -615,10 +621,10 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
                 hb = sq > m2 ? hhg : (sq < m2 ? hlg : ((hlg & 1) ? hhg : hlg));
               } else {
                 const double n64 = sqrt(sq);
-                if (n64 > 65504.0) ovf = 1;
+                if (n64 > 65504.0 && tok_ok) ovf = 1;
                 hb = __half_as_ushort(__double2half(n64 > 65504.0 ? 65504.0 : n64));
               }
-              *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb;
+              if (tile_ok) *reinterpret_cast<uint16_t*>(tile_base + norm_off + g * 128 + npos) = hb;
             }
           }
         }
@@ -705,10 +711,10 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kSEmpty + par));  // scales and flags read
-      uint8_t* dst = a.packed +
-                     ((size_t)head * a.n_tiles + (size_t)((a.mt0 + t) * 2 + hc)) * a.tile_bytes +
-                     dst_off;
-      pack_store(A, L, side, partner_xor, dst, w > 0);
+      const int64_t ptile = (a.mt0 + t) * 2 + hc;
+      const bool tile_ok = ptile * kTile < len;
+      uint8_t* dst = tile_ok ? a.sm.tile(a.packed, head, ptile) + dst_off : nullptr;
+      pack_store(A, L, side, partner_xor, dst, w > 0 && tile_ok);
     }
   }
   if (failed) atomicOr(a.status, kStatusTimeout);
@@ -833,7 +839,8 @@ cudaError_t build_code_lut(const float* thr, uint8_t* blob, cudaStream_t s) {
 // Quantize MMA tiles [mt0, mt1) of every head (keys and values in one launch).
 // Returns cudaErrorNotSupported when the inputs cannot be described by a tensor map.
 cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, const int64_t* st,
-                               int64_t mt0, int64_t mt1, uint8_t* packed, cudaStream_t s) {
+                               int64_t mt0, int64_t mt1, uint8_t* packed, const SeqMap& sm,
+                               cudaStream_t s) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap maps[2];
@@ -868,6 +875,8 @@ cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, 
   a.mt0 = mt0;
   a.mt1 = mt1;
   a.status = p->d_status;
+  a.sm = sm;
+  a.cap = p->cfg.t_capacity;
   const int64_t n_mt = mt1 - mt0;
   // SMs per head are shared between the roles by their measured cost per tile
   // (a key tile costs about twice a value tile); every CTA keeps one head

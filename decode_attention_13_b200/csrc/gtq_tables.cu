@@ -235,6 +235,9 @@ int tables_for(int device, uint64_t seed, Tables* out) {
   std::vector<double> rv64((size_t)kD * kD);
   make_rotation(seed, 0x56, kD, rv64.data());
   std::vector<float> rv(rv64.begin(), rv64.end());
+  std::vector<float> rvt((size_t)kD * kD);
+  for (int r = 0; r < kD; ++r)
+    for (int d = 0; d < kD; ++d) rvt[(size_t)d * kD + r] = rv[(size_t)r * kD + d];
   std::vector<double> dist(GTQ_MAX_BITS + 1);
   std::vector<float> thr(kThrEntries);
   std::vector<__half> lhi(kLutEntries), llo(kLutEntries);
@@ -283,6 +286,7 @@ int tables_for(int device, uint64_t seed, Tables* out) {
   if (cudaSetDevice(device) != cudaSuccess) return GTQ_ERR_CUDA;
   cudaError_t e = up((void**)&t.rot_k, rk.data(), rk.size() * sizeof(double));
   if (e == cudaSuccess) e = up((void**)&t.rot_v, rv.data(), rv.size() * sizeof(float));
+  if (e == cudaSuccess) e = up((void**)&t.rot_vt, rvt.data(), rvt.size() * sizeof(float));
   if (e == cudaSuccess) e = up((void**)&t.dist, dist.data(), dist.size() * sizeof(double));
   if (e == cudaSuccess) e = up((void**)&t.thr, thr.data(), thr.size() * sizeof(float));
   if (e == cudaSuccess) e = up((void**)&t.dec_image, img.data(), img.size() * sizeof(uint32_t));

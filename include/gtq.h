@@ -168,6 +168,61 @@ GTQ_API int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_d
 GTQ_API int gtq_decode_attn(gtq_plan* plan, const void* packed_dev, int64_t T,
                     const void* q_dev, int32_t q_dtype, float* out_dev, void* stream);
 
+/* ---- batches of sequences of their own lengths; paged caches ------------ */
+
+/*
+ * How the sequences of a batch are laid out (the page's serving setting of
+ * Abstract, with requests of different lengths; a layout of this library's own).
+ *   seq_lens_dev     device int32 [batch]: tokens held by sequence b (values
+ *                    above the call's T are clamped to T, below 0 to 0), or
+ *                    NULL: every sequence holds the call's T tokens.
+ *   block_table_dev  device int32 [batch][max_blocks], or NULL: the packed
+ *                    cache is contiguous, as gtq_packed_bytes describes.  With a
+ *                    table, the packed buffer is a pool of pages; a page holds
+ *                    one 64-token tile of every KV head of one sequence, and
+ *                    tile n of head (b, h) sits at byte offset
+ *                        ((block_table[b][n] * n_kv_heads + h) * tile_bytes)
+ *                    of the pool (tile_bytes = gtq_layout_tile_bytes).  Every
+ *                    entry a call touches (tiles below ceil(len_b / 64)) must
+ *                    name a page inside the pool; the library does not read
+ *                    the table on the host and cannot check it.
+ *   max_blocks       columns of the block table (>= 1 with a table).
+ * Both arrays are read by the kernels, on the call's stream, in stream order.
+ */
+typedef struct gtq_seq_layout {
+  const int32_t* seq_lens_dev;
+  const int32_t* block_table_dev;
+  int64_t max_blocks;
+} gtq_seq_layout;
+
+/* gtq_alloc_bits with per-sequence lengths: E_i of sequence b is the mean over
+ * its own first len_b tokens (0 for an empty sequence, whose greedy then gives
+ * every bit to the lowest eligible block: ties go to the lower index).  lay may
+ * be NULL.  Errors as gtq_alloc_bits. */
+GTQ_API int gtq_alloc_bits_ex(const gtq_config* cfg, const void* k_dev, int64_t T,
+                              const int64_t k_strides[4], const gtq_seq_layout* lay,
+                              void* stream, gtq_plan** out);
+
+/* gtq_quantize_pack into a layout: tokens [t0, t0 + n_tokens) of sequence b
+ * are written only below len_b; with a block table the tiles go to the pool's
+ * pages (packed_bytes = the pool's size, checked only against one page).
+ * t0 = GTQ_T0_TAIL writes the last n_tokens tokens of every sequence instead,
+ * [max(0, len_b - n_tokens), len_b) -- a batched decode-time append where each
+ * sequence has grown to its own length (needs seq_lens_dev).  lay may be NULL
+ * otherwise.  Errors as gtq_quantize_pack. */
+#define GTQ_T0_TAIL (-1)
+GTQ_API int gtq_quantize_pack_ex(gtq_plan* plan, const void* k_dev, const void* v_dev,
+                                 const int64_t strides[4], int64_t t0, int64_t n_tokens,
+                                 void* packed_dev, size_t packed_bytes,
+                                 const gtq_seq_layout* lay, void* stream);
+
+/* gtq_decode_attn over a layout: sequence b attends to its first len_b tokens
+ * (T is an upper bound, <= t_capacity, that sizes the launch; a sequence of
+ * length 0 gets a zero output).  lay may be NULL.  Errors as gtq_decode_attn. */
+GTQ_API int gtq_decode_attn_ex(gtq_plan* plan, const void* packed_dev, int64_t T,
+                               const gtq_seq_layout* lay, const void* q_dev, int32_t q_dtype,
+                               float* out_dev, void* stream);
+
 /* gtq_free -- release the plan and its device memory.  Synchronises the plan's
  * device (cudaFree).  NULL is accepted.  Returns GTQ_OK or GTQ_ERR_CUDA. */
 GTQ_API int gtq_free(gtq_plan* plan);

@@ -142,3 +142,15 @@ def write_head(bits, key_groups: list, vcodes: np.ndarray, vnorm16: np.ndarray, 
         kn = padrows(np.asarray(n16, np.float16))[(tok + nmap[None, :])]
         out[:n, o + 128 + gi * 128:o + 256 + gi * 128] = kn.view(np.uint8).reshape(n, 128)
     return out.ravel()
+
+
+def gather_paged_head(pool: np.ndarray, table_row, hkv: int, h: int, n_tiles: int,
+                      tb: int) -> np.ndarray:
+    """The n_tiles tiles of KV head h of one sequence, read from a paged pool
+    (page p holds one tile of every KV head: head h at (p * hkv + h) tiles),
+    concatenated in token order as a contiguous head buffer."""
+    out = np.empty(n_tiles * tb, np.uint8)
+    for n in range(n_tiles):
+        off = (int(table_row[n]) * hkv + h) * tb
+        out[n * tb:(n + 1) * tb] = pool[off:off + tb]
+    return out
