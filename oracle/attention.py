@@ -77,3 +77,38 @@ def logit_mae(q: np.ndarray, k: np.ndarray, k_hat: np.ndarray) -> float:
     q = np.asarray(q, dtype=np.float64)
     return float(np.mean(np.abs(q @ np.asarray(k_hat, np.float64).T
                                 - q @ np.asarray(k, np.float64).T)))
+
+
+def decode_general(q: np.ndarray, key_groups: list, values=None, v_fp16=None,
+                   k_recent=None, v_recent=None, seed: int = 0) -> np.ndarray:
+    """Decode over coded keys with either coded values or fp16 values (the
+    page's K-only quantization, Abstract), plus an optional window of recent
+    tokens kept in fp16 (the fp16 recent-key buffer the page's method does
+    without, Abstract).
+
+    Reading taken: the query attends to the T coded tokens and then to the W
+    window tokens in one softmax; window logits are q . k / sqrt(d) with the
+    exact fp16 keys, window values are the exact fp16 values.  With K-only
+    values, P.V uses the T exact fp16 value rows (no rotation).  Returns [G, d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    G, d = q.shape
+    T = (values.codes.shape[0] if values is not None else np.asarray(v_fp16).shape[0])
+    s = np.zeros((G, T))
+    for g in key_groups:
+        r = rotation.key_rotation(g.m, seed)
+        qg = q[:, list(g.coords)] @ r.T
+        cb = lloyd_max.decode(g.codes, g.width)
+        s += (qg @ cb.T) * (g.norm16.astype(np.float64) / np.sqrt(g.m))[None, :]
+    s /= np.sqrt(d)
+    if values is not None:
+        cbv = lloyd_max.decode(values.codes, values.width)
+        v_rows = (cbv * (values.norm16.astype(np.float64) / np.sqrt(d))[:, None]) \
+            @ rotation.value_rotation(d, seed)                      # R_V^T per row
+    else:
+        v_rows = np.asarray(v_fp16, dtype=np.float64)
+    if k_recent is not None and len(k_recent):
+        kr = np.asarray(k_recent, dtype=np.float64)
+        s = np.concatenate([s, q @ kr.T / np.sqrt(d)], axis=1)
+        v_rows = np.concatenate([v_rows, np.asarray(v_recent, dtype=np.float64)], axis=0)
+    return _softmax(s) @ v_rows

@@ -62,3 +62,53 @@ def test_block_gtq_logit_mae_not_above_uniform(kb):
         assert mae_b <= mae_u
         ratios.append(mae_b / mae_u)
     print("Block-GTQ / uniform logit MAE at K%d:" % kb, np.round(ratios, 3))
+
+
+def test_general_reduces_to_rotated_without_window():
+    hd, bits, kg, vg = _coded((25,), 300, 4, 3, 3)
+    a = attention.decode_general(hd["q"], kg, values=vg)
+    b = attention.decode_rotated(hd["q"], kg, vg)
+    assert np.max(np.abs(a - b)) < 1e-12 * max(1.0, np.max(np.abs(b)))
+    c = attention.decode_general(hd["q"], kg, values=vg, k_recent=np.zeros((0, 128)),
+                                 v_recent=np.zeros((0, 128)))
+    assert np.max(np.abs(c - b)) < 1e-12 * max(1.0, np.max(np.abs(b)))
+
+
+def test_key_only_matches_textbook_attention_on_dequantised_keys():
+    # second route: rebuild k_hat in the original basis, textbook softmax with exact V
+    hd, bits, kg, vg = _coded((26,), 333, 3, 3, 3)
+    a = attention.decode_general(hd["q"], kg, v_fp16=hd["v"])
+    k_hat = quantize.dequantize_keys(kg, 128, 333)
+    q = hd["q"].astype(np.float64)
+    s = q @ k_hat.T / np.sqrt(128)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    b = p @ hd["v"].astype(np.float64)
+    assert np.max(np.abs(a - b)) < 1e-12 * max(1.0, np.max(np.abs(b)))
+
+
+def test_window_holding_every_token_is_exact_attention():
+    hd = synth.head((27,), T=200, d=128, theta=1e4, g_q=4, dtype=np.float16)
+    empty = quantize.quantize_keys(hd["k"][:0], np.full(64, 3), rope.HALF)
+    a = attention.decode_general(hd["q"], empty, v_fp16=hd["v"][:0], k_recent=hd["k"],
+                                 v_recent=hd["v"])
+    ex = attention.attention_exact(hd["q"], hd["k"], hd["v"])
+    assert np.max(np.abs(a - ex)) < 1e-12 * max(1.0, np.max(np.abs(ex)))
+
+
+def test_window_after_coded_tokens_is_one_softmax():
+    # coded prefix + fp16 window == textbook attention over [k_hat ; k_window]
+    hd, bits, kg_all, vg_all = _coded((28,), 260, 2, 3, 3)
+    T = 200
+    kg = quantize.quantize_keys(hd["k"][:T], bits, rope.HALF)
+    vg = quantize.quantize_values(hd["v"][:T], 3)
+    a = attention.decode_general(hd["q"], kg, values=vg, k_recent=hd["k"][T:],
+                                 v_recent=hd["v"][T:])
+    k_all = np.concatenate([quantize.dequantize_keys(kg, 128, T), hd["k"][T:].astype(np.float64)])
+    v_all = np.concatenate([quantize.dequantize_values(vg), hd["v"][T:].astype(np.float64)])
+    q = hd["q"].astype(np.float64)
+    s = q @ k_all.T / np.sqrt(128)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    b = p @ v_all
+    assert np.max(np.abs(a - b)) < 1e-12 * max(1.0, np.max(np.abs(b)))
