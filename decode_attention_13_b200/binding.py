@@ -46,7 +46,7 @@ ABI_FUNCTIONS = (
     "gtq_free", "gtq_packed_bytes", "gtq_get_bits", "gtq_get_energy", "gtq_status",
     "gtq_strerror", "gtq_last_error", "gtq_lloyd_max", "gtq_rotation", "gtq_layout_tile_bytes",
     "gtq_block_energy_noalloc", "gtq_plan_device_bytes", "gtq_raise_status",
-    "gtq_alloc_bits_ex", "gtq_quantize_pack_ex", "gtq_decode_attn_ex",
+    "gtq_alloc_bits_ex", "gtq_quantize_pack_ex", "gtq_decode_attn_ex", "gtq_decode_attn_full",
 )
 
 
@@ -90,6 +90,36 @@ def seq_layout(seq_lens=None, block_table=None):
     return lay
 
 
+class gtq_fp16_kv(ctypes.Structure):
+    _fields_ = [
+        ("v_dev", ctypes.c_void_p), ("v_strides", ctypes.c_int64 * 4),
+        ("recent_k_dev", ctypes.c_void_p), ("recent_v_dev", ctypes.c_void_p),
+        ("recent_strides", ctypes.c_int64 * 4), ("recent_lens_dev", ctypes.c_void_p),
+        ("recent_len", ctypes.c_int64),
+    ]
+
+
+def fp16_kv(v=None, recent_k=None, recent_v=None, recent_lens=None, recent_len=None):
+    """A gtq_fp16_kv from device fp16 tensors: values [batch, kv_heads, tokens, 128]
+    of a K-only plan, and a window of recent keys / values [batch, kv_heads, rows,
+    128] (same strides for both) with optional int32 lengths [batch].  Keep the
+    tensors alive while the calls that use it run."""
+    kv = gtq_fp16_kv()
+    if v is not None:
+        kv.v_dev = _ptr(v)
+        kv.v_strides = (ctypes.c_int64 * 4)(*[int(s) for s in v.stride()])
+    if recent_k is not None:
+        if tuple(recent_k.stride()) != tuple(recent_v.stride()):
+            raise ValueError("recent keys and values must share strides")
+        kv.recent_k_dev = _ptr(recent_k)
+        kv.recent_v_dev = _ptr(recent_v)
+        kv.recent_strides = (ctypes.c_int64 * 4)(*[int(s) for s in recent_k.stride()])
+        kv.recent_len = int(recent_k.shape[2]) if recent_len is None else int(recent_len)
+    if recent_lens is not None:
+        kv.recent_lens_dev = _ptr(recent_lens)
+    return kv
+
+
 def make_config(batch, n_q_heads, n_kv_heads, k_bits, v_bits, t_capacity, head_dim=128,
                 max_bits=8, rope_pairing=PAIRING_HALF, in_dtype=DTYPE_FP16, seed=0) -> gtq_config:
     return gtq_config(batch, n_q_heads, n_kv_heads, head_dim, k_bits, v_bits, max_bits,
@@ -126,6 +156,8 @@ def _load():
         "gtq_quantize_pack_ex": (I32, [P, P, P, I64x4, I64, I64, P, SZ,
                                        ctypes.POINTER(gtq_seq_layout), P]),
         "gtq_decode_attn_ex": (I32, [P, P, I64, ctypes.POINTER(gtq_seq_layout), P, I32, P, P]),
+        "gtq_decode_attn_full": (I32, [P, P, I64, ctypes.POINTER(gtq_seq_layout),
+                                       ctypes.POINTER(gtq_fp16_kv), P, I32, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -270,6 +302,18 @@ def gtq_decode_attn_ex(plan: Plan, packed, T: int, q, out, layout=None, stream=N
     rc = _lib.gtq_decode_attn_ex(plan.handle, _ptr(packed), int(T), _lay(layout), _ptr(q),
                                  int(q_dtype), _ptr(out), _stream(stream))
     _check(rc, "gtq_decode_attn_ex")
+
+
+def gtq_decode_attn_full(plan: Plan, packed, T: int, q, out, layout=None, kv=None, stream=None,
+                         q_dtype=None) -> None:
+    if q_dtype is None:
+        import torch
+
+        q_dtype = DTYPE_FP32 if q.dtype == torch.float32 else DTYPE_FP16
+    rc = _lib.gtq_decode_attn_full(plan.handle, _ptr(packed), int(T), _lay(layout),
+                                   None if kv is None else ctypes.byref(kv), _ptr(q),
+                                   int(q_dtype), _ptr(out), _stream(stream))
+    _check(rc, "gtq_decode_attn_full")
 
 
 def gtq_free(plan: Plan) -> None:

@@ -23,7 +23,7 @@ int check_config(const gtq_config* c, bool need_128) {
   if (need_128 && c->head_dim != kD) return GTQ_ERR_UNSUPPORTED;
   if (c->max_bits < 1 || c->max_bits > GTQ_MAX_BITS) return GTQ_ERR_INVALID;
   if (c->k_bits < 1 || c->k_bits > c->max_bits) return GTQ_ERR_INVALID;
-  if (c->v_bits < 1 || c->v_bits > GTQ_MAX_BITS) return GTQ_ERR_INVALID;
+  if (c->v_bits < 0 || c->v_bits > GTQ_MAX_BITS) return GTQ_ERR_INVALID;  // 0: K-only
   if (c->rope_pairing != GTQ_PAIRING_HALF && c->rope_pairing != GTQ_PAIRING_INTERLEAVED)
     return GTQ_ERR_INVALID;
   if (c->in_dtype != GTQ_DTYPE_FP16 && c->in_dtype != GTQ_DTYPE_FP32) return GTQ_ERR_INVALID;
@@ -138,8 +138,8 @@ int record_cuda_error(cudaError_t e) { return cuda_code(e); }
 extern "C" {
 
 size_t gtq_layout_tile_bytes(int32_t k_bits, int32_t v_bits) {
-  if (k_bits < 1 || k_bits > GTQ_MAX_BITS || v_bits < 1 || v_bits > GTQ_MAX_BITS) return 0;
-  return (size_t)1024 * (k_bits + v_bits) + 128 + 128 * kMaxGroups;
+  if (k_bits < 1 || k_bits > GTQ_MAX_BITS || v_bits < 0 || v_bits > GTQ_MAX_BITS) return 0;
+  return (size_t)key_norm_offset(k_bits, v_bits) + 128 * kMaxGroups;
 }
 
 int gtq_alloc_bits(const gtq_config* cfg, const void* k_dev, int64_t T, const int64_t k_strides[4],
@@ -205,7 +205,10 @@ int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_dev,
 int gtq_quantize_pack_ex(gtq_plan* plan, const void* k_dev, const void* v_dev,
                          const int64_t strides[4], int64_t t0, int64_t n_tokens, void* packed_dev,
                          size_t packed_bytes, const gtq_seq_layout* lay, void* stream) {
-  if (!plan || !k_dev || !v_dev || !strides || !packed_dev) return GTQ_ERR_INVALID;
+  if (!plan || !k_dev || !strides || !packed_dev) return GTQ_ERR_INVALID;
+  // values: coded plans need them, K-only plans (v_bits 0) take none
+  if ((v_dev != nullptr) != (plan->cfg.v_bits > 0)) return GTQ_ERR_INVALID;
+  if (!v_dev) v_dev = k_dev;  // (never read)
   if (plan->cfg.head_dim != kD) return GTQ_ERR_UNSUPPORTED;
   const bool tail = t0 == GTQ_T0_TAIL;
   if (tail && !(lay && lay->seq_lens_dev)) return GTQ_ERR_INVALID;
@@ -234,7 +237,37 @@ int gtq_decode_attn(gtq_plan* plan, const void* packed_dev, int64_t T, const voi
 int gtq_decode_attn_ex(gtq_plan* plan, const void* packed_dev, int64_t T,
                        const gtq_seq_layout* lay, const void* q_dev, int32_t q_dtype,
                        float* out_dev, void* stream) {
+  return gtq_decode_attn_full(plan, packed_dev, T, lay, nullptr, q_dev, q_dtype, out_dev, stream);
+}
+
+int gtq_decode_attn_full(gtq_plan* plan, const void* packed_dev, int64_t T,
+                         const gtq_seq_layout* lay, const gtq_fp16_kv* kv, const void* q_dev,
+                         int32_t q_dtype, float* out_dev, void* stream) {
   if (!plan || !packed_dev || !q_dev || !out_dev) return GTQ_ERR_INVALID;
+  Fp16Kv f;
+  const bool konly = plan->cfg.v_bits == 0;
+  if (konly != (kv && kv->v_dev)) return GTQ_ERR_INVALID;  // values: coded xor fp16
+  if (konly) {
+    if (!aligned(kv->v_dev, 16) || kv->v_strides[3] != 1) return GTQ_ERR_INVALID;
+    for (int i = 0; i < 3; ++i)
+      if (kv->v_strides[i] < 0 || kv->v_strides[i] % 8) return GTQ_ERR_INVALID;
+    f.v = (const __half*)kv->v_dev;
+    for (int i = 0; i < 4; ++i) f.vs[i] = kv->v_strides[i];
+  }
+  if (kv && kv->recent_len != 0) {
+    if (kv->recent_len < 0 || kv->recent_len > kMaxWindow) return GTQ_ERR_INVALID;
+    if (!kv->recent_k_dev || !kv->recent_v_dev || !aligned(kv->recent_k_dev, 8) ||
+        !aligned(kv->recent_v_dev, 8) || kv->recent_strides[3] != 1 ||
+        !aligned(kv->recent_lens_dev, 4))
+      return GTQ_ERR_INVALID;
+    for (int i = 0; i < 3; ++i)
+      if (kv->recent_strides[i] < 0 || kv->recent_strides[i] % 4) return GTQ_ERR_INVALID;
+    f.rk = (const __half*)kv->recent_k_dev;
+    f.rv = (const __half*)kv->recent_v_dev;
+    for (int i = 0; i < 4; ++i) f.rs[i] = kv->recent_strides[i];
+    f.rlens = kv->recent_lens_dev;
+    f.rlen = kv->recent_len;
+  }
   if (plan->cfg.head_dim != kD) return GTQ_ERR_UNSUPPORTED;
   if (T < 1 || T > plan->cfg.t_capacity) return GTQ_ERR_INVALID;
   if (q_dtype != GTQ_DTYPE_FP16 && q_dtype != GTQ_DTYPE_FP32) return GTQ_ERR_INVALID;
@@ -242,7 +275,7 @@ int gtq_decode_attn_ex(gtq_plan* plan, const void* packed_dev, int64_t T,
     return GTQ_ERR_INVALID;
   if (check_layout(lay, T) != GTQ_OK) return GTQ_ERR_INVALID;
   return cuda_code(launch_decode(plan, (const uint8_t*)packed_dev, T, q_dev, q_dtype, out_dev,
-                                 seq_map(plan, lay), (cudaStream_t)stream));
+                                 seq_map(plan, lay), f, (cudaStream_t)stream));
 }
 
 int gtq_free(gtq_plan* plan) {

@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kAThreads) append_kernel(AppendArgs a) {
       }
     }
     // norms: thread (token j, group gi)
-    const int knorm_off = 1024 * (a.kb + a.vb) + 128;
+    const int knorm_off = key_norm_offset(a.kb, a.vb);
     for (int i = tid; i < n * m.n_groups; i += kAThreads) {
       const int j = i / m.n_groups, gi = i % m.n_groups;
       const int64_t t = t0 + j;
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kAThreads) append_kernel(AppendArgs a) {
     }
     const float sqrt_d = sqrtf((float)kD);
     const int i16 = p >> 4, g = p & 7, hd = (p >> 3) & 1;  // dim tile, row, upper half
-    const int vcode_off = 1024 * a.kb, vnorm_off = 1024 * (a.kb + a.vb);
+    const int vcode_off = 1024 * a.kb, vnorm_off = value_norm_offset(a.kb, a.vb);
 #pragma unroll
     for (int j = 0; j < kAppendMax; ++j) {
       if (j >= n) break;
@@ -303,7 +303,7 @@ cudaError_t launch_append(const gtq_plan* p, const void* k, const void* v, const
   a.status = p->d_status;
   a.sm = sm;
   a.cap = p->cfg.t_capacity;
-  const dim3 grid((unsigned)p->n_heads, 2);
+  const dim3 grid((unsigned)p->n_heads, p->cfg.v_bits > 0 ? 2 : 1);  // K-only: keys alone
   cudaError_t e;
   if (p->cfg.in_dtype == GTQ_DTYPE_FP16) {
     e = cudaFuncSetAttribute(append_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,

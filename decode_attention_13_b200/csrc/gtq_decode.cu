@@ -26,10 +26,19 @@
 //            16 splits merges the group (and fetches R_V), the last group
 //            merges the rest and writes o = R_V^T o_rot / l.  Tickets and the
 //            tile counter return to 0 for the next call.
+// K-only plans (values kept in fp16, the page's K-only quantization, Abstract)
+// take decode_kernel<0>: each stage also receives the tiles' fp16 value rows
+// by a tensor copy (128-byte swizzle, so that the transposing ldmatrix that
+// forms A = V^T is free of bank conflicts), P.V runs in the original basis and
+// no R_V^T product follows.  An fp16 window of recent tokens (the recent-key
+// buffer the page's method does without, Abstract) is attended by split 0 on
+// the CUDA cores into a partial of its own, combined with the cache's (m, l)
+// by the CTA that finishes the head.
 #include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstddef>
+#include <cstring>
 
 #include "gtq_internal.h"
 
@@ -89,6 +98,17 @@ struct DecodeArgs {
   int prefetch;       // tiles this CTA prefetches into L2 before the dependency wait
   int64_t static_per; // tiles [split * static_per, +static_per) are this CTA's; the rest
                       // (from splits * static_per on) go out through the tile counter
+  // K-only plans
+  int voff;           // bytes of a stage before its value rows (kTPS x 16 KB, swizzled)
+  int v_loads;        // tensor copies per tile: 1 (5-D map) or 2 (4-D map, one per half)
+  const __half* v16;  // fp16 values (L2 prefetch only; the copies go through the map)
+  int64_t vs0, vs1, vs2;  // their strides in elements
+  // fp16 window of recent tokens
+  const __half* rk;
+  const __half* rv;
+  int64_t rs0, rs1, rs2;
+  const int32_t* rlens;
+  int rlen;           // rows per head, 0: no window
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -124,6 +144,30 @@ __device__ __forceinline__ void bulk_copy_hint(void* dst, const void* src, unsig
       : "memory");
 }
 // bring bytes into L2 (no effect on the values any load returns)
+// tensor copies of value rows into shared memory (no cluster multicast)
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, int c4, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
 __device__ __forceinline__ void prefetch_l2(const void* src, unsigned bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
@@ -431,7 +475,8 @@ __device__ bool arrive_last(unsigned* ticket, unsigned count, int* flag) {
 // once; the two parities combine through `scratch` (shared, 2 x 8 x
 // kPartialStride floats).  Partials come from other CTAs: loads bypass L1.
 __device__ __noinline__ void merge_partials(const float* head_parts, int first, int count,
-                                            float* dst, float (*o_rot)[kD], float* scratch) {
+                                            float* dst, float (*o_rot)[kD], float* scratch,
+                                            float* hm, float* hl) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   for (int item = warp; item < 16; item += nwarps) {
     const int hh = item >> 1, sub = item & 1;
@@ -486,6 +531,10 @@ __device__ __noinline__ void merge_partials(const float* head_parts, int first, 
       const float inv = L > 0.f ? 1.f / L : 0.f;
       *reinterpret_cast<float4*>(&o_rot[hh][4 * d4]) =
           make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      if (d4 == 0) {  // (M, L) of the whole cache, for the window's combination
+        hm[hh] = M;
+        hl[hh] = L;
+      }
     }
   }
 }
@@ -504,13 +553,114 @@ struct HeadView {
   }
 };
 
+// Partial (m, l, o) of the 8 query heads over the sequence's fp16 window rows,
+// with logits in base 2 like the cache's (log2(e) q.k / sqrt(d)).  The consumer
+// warps take rows in turn (lane = 4 dims, one online softmax per warp); the
+// warps then merge through shared memory and the result is written to dst in
+// the layout of a split's partial.  Every thread of the CTA calls it.
+struct WindowArgs {
+  const void* q;
+  const __half* rk;
+  const __half* rv;
+  int64_t rs0, rs1, rs2;
+  const int32_t* rlens;
+  int rlen, q_fp32, hkv, gq;
+};
+__device__ __noinline__ void window_partial(const WindowArgs a, DecodeSmem& s, int b, int h,
+                                            int ncw, float* dst, float* wo) {
+  __syncthreads();  // wo and the warp scales are free
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t wl = a.rlens ? min(max((int64_t)a.rlens[b], (int64_t)0), (int64_t)a.rlen)
+                             : (int64_t)a.rlen;
+  if (warp < ncw) {
+    float qv[8][4], m[8], l[8], o[8][4];
+    const float qs = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = 0.f;
+        if (hh < a.gq) {
+          const size_t qi = (((size_t)b * a.hkv + h) * a.gq + hh) * kD + 4 * lane + e;
+          v = a.q_fp32 ? reinterpret_cast<const float*>(a.q)[qi]
+                       : __half2float(reinterpret_cast<const __half*>(a.q)[qi]);
+        }
+        qv[hh][e] = v * qs;
+        o[hh][e] = 0.f;
+      }
+      m[hh] = -1e30f;
+      l[hh] = 0.f;
+    }
+    const __half* kr = a.rk + b * a.rs0 + h * a.rs1 + 4 * lane;
+    const __half* vr = a.rv + b * a.rs0 + h * a.rs1 + 4 * lane;
+    for (int64_t r = warp; r < wl; r += ncw) {
+      const uint2 kq = __ldg(reinterpret_cast<const uint2*>(kr + r * a.rs2));
+      const uint2 vq = __ldg(reinterpret_cast<const uint2*>(vr + r * a.rs2));
+      const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kq.x));
+      const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kq.y));
+      const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vq.x));
+      const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vq.y));
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) {
+        float sc = qv[hh][0] * k01.x;
+        sc = fmaf(qv[hh][1], k01.y, sc);
+        sc = fmaf(qv[hh][2], k23.x, sc);
+        sc = fmaf(qv[hh][3], k23.y, sc);
+#pragma unroll
+        for (int x = 16; x >= 1; x >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, x);
+        const float mn = fmaxf(m[hh], sc), al = exp2f(m[hh] - mn), p = exp2f(sc - mn);
+        l[hh] = fmaf(l[hh], al, p);
+        o[hh][0] = fmaf(o[hh][0], al, p * v01.x);
+        o[hh][1] = fmaf(o[hh][1], al, p * v01.y);
+        o[hh][2] = fmaf(o[hh][2], al, p * v23.x);
+        o[hh][3] = fmaf(o[hh][3], al, p * v23.y);
+        m[hh] = mn;
+      }
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) {
+        s.wm[warp][hh] = m[hh];
+        s.wl[warp][hh] = l[hh];
+      }
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) wo[(warp * kD + 4 * lane + e) * 8 + hh] = o[hh][e];
+  }
+  __syncthreads();
+  if (tid < 8) {
+    const int hh = tid;
+    float M = -1e30f;
+    for (int w = 0; w < ncw; ++w) M = fmaxf(M, s.wm[w][hh]);
+    float L = 0.f;
+    for (int w = 0; w < ncw; ++w) {
+      const float sc = exp2f(s.wm[w][hh] - M);
+      s.wsc[w][hh] = sc;
+      L = fmaf(sc, s.wl[w][hh], L);
+    }
+    *reinterpret_cast<float2*>(dst + hh * kPartialStride) = make_float2(M, L);
+  }
+  __syncthreads();
+  for (int idx = tid; idx < 8 * kD; idx += blockDim.x) {
+    const int hh = idx & 7, d = idx >> 3;
+    float v = 0.f;
+    for (int w = 0; w < ncw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * kD + d) * 8 + hh], v);
+    dst[hh * kPartialStride + 4 + d] = v;
+  }
+}
+
 template <int VB>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap vmap, DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem& s = *reinterpret_cast<DecodeSmem*>(smem_raw);
   const uint32_t raw_sa = smem_u32(smem_raw);
   uint8_t* tab = smem_raw + (kTabSharedAddr - raw_sa);
-  const uint32_t stage_sa = (raw_sa + (uint32_t)sizeof(DecodeSmem) + 127u) & ~127u;
+  // value rows (K-only plans) land with the 128-byte swizzle: 1024-byte stages
+  constexpr uint32_t kStageAlign = VB > 0 ? 128u : 1024u;
+  const uint32_t stage_sa =
+      (raw_sa + (uint32_t)sizeof(DecodeSmem) + kStageAlign - 1) & ~(kStageAlign - 1);
   uint8_t* stages = smem_raw + (stage_sa - raw_sa);
   const int area = (int)(kTabSharedAddr - stage_sa);  // bytes of the stage area
   float* pack = reinterpret_cast<float*>(stages + area - kPackArea);  // rotation pack at setup
@@ -558,11 +708,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     const int64_t tiles = (min(max(Tp, (int64_t)0), a.T) + kTile - 1) / kTile;
     const int64_t t0 = (int64_t)split * a.static_per;
     const int64_t n = min((int64_t)a.prefetch, tiles - t0);
-    if (n > 0) prefetch_l2(hv.tile(a.packed, t0), (unsigned)(n * a.tile_bytes));
+    const int64_t Tc = min(max(Tp, (int64_t)0), a.T);
+    // value rows [t0, t0 + n tiles) below the sequence's length, when contiguous
+    auto prefetch_values = [&](int64_t tt0, int64_t nt) {
+      if (VB > 0 || a.vs2 != kD) return;
+      const int64_t r0 = tt0 * kTile, r1 = min((tt0 + nt) * kTile, Tc);
+      if (r1 > r0)
+        prefetch_l2(a.v16 + b * a.vs0 + h * a.vs1 + r0 * kD, (unsigned)((r1 - r0) * kD * 2));
+    };
+    if (n > 0) {
+      prefetch_l2(hv.tile(a.packed, t0), (unsigned)(n * a.tile_bytes));
+      prefetch_values(t0, n);
+    }
     const int64_t dyn0 = (int64_t)nsplit * a.static_per;
     const int64_t dper = (tiles - dyn0 + nsplit - 1) / nsplit;
     const int64_t d0 = dyn0 + (int64_t)split * dper, dn = min(dper, tiles - d0);
-    if (dper > 0 && dn > 0) prefetch_l2(hv.tile(a.packed, d0), (unsigned)(dn * a.tile_bytes));
+    if (dper > 0 && dn > 0) {
+      prefetch_l2(hv.tile(a.packed, d0), (unsigned)(dn * a.tile_bytes));
+      prefetch_values(d0, dn);
+    }
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -592,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       if (!__all_sync(0xffffffffu, mbar_wait(&s.meta_bar, 0))) {
         failed = true;
       } else {
-        const int load_bytes = 1024 * (a.kb + VB) + 128 + 128 * s.meta.n_groups;
+        const int load_bytes = key_norm_offset(a.kb, VB) + 128 * s.meta.n_groups;
         const int pack_lo = area - kPackArea;
         const uint64_t pol = evict_first_policy();
         unsigned* ctr = head_tickets + kSchedWord;
@@ -651,16 +815,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
             }
             if (lane == 0) {
               s.stage_tile[slot] = make_int2((int)t0, (int)t1);
+              // K-only: 16 KB of fp16 value rows per tile (zero past the call's T)
+              const unsigned vbytes = VB > 0 ? 0u : (t1 >= 0 ? 2u : 1u) * (unsigned)(kTile * kD * 2);
               if (t1 >= 0 && !hv.pages) {  // adjacent tiles: one copy
-                mbar_expect_tx(&s.full[slot], (unsigned)(a.tile_bytes + load_bytes));
+                mbar_expect_tx(&s.full[slot], (unsigned)(a.tile_bytes + load_bytes) + vbytes);
                 bulk_copy_hint(dst, hv.tile(a.packed, t0), (unsigned)(a.tile_bytes + load_bytes),
                                &s.full[slot], pol);
               } else {
-                mbar_expect_tx(&s.full[slot], (unsigned)(t1 >= 0 ? 2 * load_bytes : load_bytes));
+                mbar_expect_tx(&s.full[slot],
+                               (unsigned)(t1 >= 0 ? 2 * load_bytes : load_bytes) + vbytes);
                 bulk_copy_hint(dst, hv.tile(a.packed, t0), (unsigned)load_bytes, &s.full[slot], pol);
                 if (t1 >= 0)
                   bulk_copy_hint(dst + a.tile_bytes, hv.tile(a.packed, t1), (unsigned)load_bytes,
                                  &s.full[slot], pol);
+              }
+              if (VB == 0) {
+                // rows of tile tt: box (64 dims, 64 tokens, both dim halves) -> [half][token][64]
+                auto load_values = [&](uint8_t* vdst, int64_t tt) {
+                  const int row = (int)(tt * kTile);
+                  if (a.v_loads == 1) {
+                    tma_load_5d(vdst, &vmap, 0, row, 0, h, b, &s.full[slot]);
+                  } else {
+                    tma_load_4d(vdst, &vmap, 0, row, h, b, &s.full[slot]);
+                    tma_load_4d(vdst + kTile * 128, &vmap, 64, row, h, b, &s.full[slot]);
+                  }
+                };
+                load_values(dst + a.voff, t0);
+                if (t1 >= 0) load_values(dst + a.voff + kTile * kD * 2, t1);
               }
             }
           } else {
@@ -789,7 +970,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
     const int n_groups = m.n_groups;
     const int kb = a.kb;
     const int load_v = 1024 * kb;
-    const int vnorm_off = 1024 * (kb + VB), knorm_off = vnorm_off + 128;
+    const int vnorm_off = value_norm_offset(kb, VB), knorm_off = key_norm_offset(kb, VB);
     TabBase tb;
     tb.bss = kTabSharedAddr;
     tb.b32 = kTabSharedAddr | ((uint32_t)lane << 2);
@@ -900,15 +1081,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
           O[i][3] *= alpha[1];
         }
       }
-      const uint2 vq = *reinterpret_cast<const uint2*>(tl + vnorm_off + g * 16 + wh * 8);
-      const __half2* vnh = reinterpret_cast<const __half2*>(&vq);
+      // coded values: p times the token's fp16 norm / sqrt(d); fp16 values: p
+      float2 vsc[2] = {make_float2(1.f, 1.f), make_float2(1.f, 1.f)};
+      if (VB > 0) {
+        const uint2 vq = *reinterpret_cast<const uint2*>(tl + vnorm_off + g * 16 + wh * 8);
+        const __half2* vnh = reinterpret_cast<const __half2*>(&vq);
+        const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          vsc[mt] = __half22float2(vnh[mt]);
+          vsc[mt].x *= inv_sqrt_d;
+          vsc[mt].y *= inv_sqrt_d;
+        }
+      }
       uint32_t PB[2][2];
-      const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128)
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        float2 vn = __half22float2(vnh[mt]);
-        vn.x *= inv_sqrt_d;
-        vn.y *= inv_sqrt_d;
+        const float2 vn = vsc[mt];
         float pp[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -922,10 +1111,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         PB[mt][1] = movmatrix_t(pack_half2(__float2half_rn(pp[2]), __float2half_rn(pp[3])));
       }
       // ---------------------------------------------------------------- P.V
-      const uint8_t* vcodes = tl + load_v;
+      if constexpr (VB > 0) {
+        const uint8_t* vcodes = tl + load_v;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        value_tile<VB>(vcodes + ((i * 8 + g) * 4 + t) * VB * 4, wh, tb, PB, O[i]);
+        for (int i = 0; i < 8; ++i)
+          value_tile<VB>(vcodes + ((i * 8 + g) * 4 + t) * VB * 4, wh, tb, PB, O[i]);
+      } else {
+        // A = V^T (16 dims x 16 tokens) by a transposing ldmatrix.x4: matrix
+        // lane >> 3 holds dims + 8 (bit 0) and tokens + 8 (bit 1); the lane
+        // gives the address of one token row, whose 16-byte chunks sit
+        // XOR-swizzled by the row's index mod 8
+        const uint32_t vrow = stage_sa + (uint32_t)(slot * a.stride + a.voff + jk * kTile * kD * 2) +
+                              (uint32_t)(32 * wh + (lane & 7) + 8 * (lane >> 4)) * 128u;
+        const uint32_t lx = (uint32_t)(((lane >> 3) & 1) ^ (lane & 7));
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu;  // rows past the sequence are zero
+          if (!full) {
+            const int64_t tk = tok0 + 16 * kk + 2 * t;
+            m0 = (tk < T ? 0xffffu : 0u) | (tk + 1 < T ? 0xffff0000u : 0u);
+            m1 = (tk + 8 < T ? 0xffffu : 0u) | (tk + 9 < T ? 0xffff0000u : 0u);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint32_t av[4];
+            ldmatrix_x4_trans(av, vrow + (uint32_t)(kk * 16 * 128 + (i >> 2) * kTile * 128) +
+                                      ((((uint32_t)(2 * i) & 7u) ^ lx) << 4));
+            av[0] &= m0;
+            av[1] &= m0;
+            av[2] &= m1;
+            av[3] &= m1;
+            mma16816(O[i], av, PB[kk][0], PB[kk][1]);
+          }
+        }
+      }
       // ---------------------------------------------------- release the stage
       advance();
     }
@@ -1001,38 +1220,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
       if (d == 0) *reinterpret_cast<float2*>(part + hh * kPartialStride) = make_float2(s.hm[hh], s.hl[hh]);
     }
   }
+  // split 0 also attends the fp16 window, before its arrival publishes it
+  float* wpart = head_parts + (size_t)kWindowSlot * 8 * kPartialStride;
+  if (a.rlen > 0 && split == 0) {
+    const WindowArgs wa = {a.q, a.rk, a.rv, a.rs0, a.rs1, a.rs2, a.rlens, a.rlen, a.q_fp32, a.hkv, a.gq};
+    window_partial(wa, s, b, h, ncw, wpart, wo);
+  }
   // ---------------- merge of the splits, without waiting: the last CTA to
   // arrive in a group of kMergeGroup splits merges the group into a
   // second-level partial, and the last group to finish merges those.  A CTA
-  // that may finish fetches R_V while it merges.
-  auto fetch_rv = [&]() {
+  // that may finish fetches R_V while it merges (coded values only).
+  auto fetch_rv = [&]() -> bool {
+    if (VB == 0) return false;
     if (tid == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_expect_tx(&s.rv_bar, (unsigned)(kD * kD * sizeof(float)));
       bulk_copy(rv, a.rot_v, kD * kD * sizeof(float), &s.rv_bar);
     }
+    return true;
   };
   bool finish = nsplit == 1, rv_issued = false;
   if (finish) {
     __syncthreads();
-    fetch_rv();
-    rv_issued = true;
+    rv_issued = fetch_rv();
   } else {
     const int n_grp = (nsplit + kMergeGroup - 1) / kMergeGroup;
     const int grp = split / kMergeGroup;
     const int n1 = min(kMergeGroup, nsplit - grp * kMergeGroup);
     if (arrive_last(&head_tickets[1 + grp], (unsigned)n1, &s.flag)) {
-      fetch_rv();
-      rv_issued = true;
+      rv_issued = fetch_rv();
       if (n_grp == 1) {
-        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qa, mscratch);
+        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qa, mscratch, s.hm, s.hl);
         finish = true;
       } else {
         merge_partials(head_parts, grp * kMergeGroup, n1,
                        head_parts + (size_t)(kMaxSplits + grp) * 8 * kPartialStride, nullptr,
-                       mscratch);
+                       mscratch, s.hm, s.hl);
         if (arrive_last(&head_tickets[0], (unsigned)n_grp, &s.flag)) {
-          merge_partials(head_parts, kMaxSplits, n_grp, nullptr, s.qa, mscratch);
+          merge_partials(head_parts, kMaxSplits, n_grp, nullptr, s.qa, mscratch, s.hm, s.hl);
           finish = true;
         }
       }
@@ -1046,6 +1271,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
   rv_ok = __syncthreads_and(rv_ok);
   if (!rv_ok) {
     if (tid == 0) atomicOr(a.status, kStatusTimeout);
+    return;
+  }
+  // out = cr o_cache + cw o_window (o_cache normalised, o_window not): the
+  // two softmax parts rescaled to their common maximum
+  if (tid < 8) {
+    float cr = 1.f, cw = 0.f;
+    if (a.rlen > 0) {
+      const float2 mlw = __ldcg(reinterpret_cast<const float2*>(wpart + tid * kPartialStride));
+      const float M = s.hm[tid], L = s.hl[tid], Mx = fmaxf(M, mlw.x);
+      const float wr = exp2f(M - Mx) * L, ww = exp2f(mlw.x - Mx);
+      const float den = fmaf(ww, mlw.y, wr);
+      cr = den > 0.f ? wr / den : 0.f;
+      cw = den > 0.f ? ww / den : 0.f;
+    }
+    s.wm[0][tid] = cr;
+    s.wl[0][tid] = cw;
+  }
+  float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
+  auto window_o = [&](int hh, int dd) -> float {
+    return a.rlen > 0 ? s.wl[0][hh] * __ldcg(wpart + hh * kPartialStride + 4 + dd) : 0.f;
+  };
+  if (VB == 0) {  // fp16 values: o_cache is already in the original basis
+    __syncthreads();
+    for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
+      const int hh = idx >> 7, dd = idx & (kD - 1);
+      out_head[idx] = fmaf(s.wm[0][hh], s.qa[hh][dd], window_o(hh, dd));
+    }
     return;
   }
   // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r]: thread = (dd pair, 16 rows r of
@@ -1078,13 +1330,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeArgs a) {
         *reinterpret_cast<float2*>(red + (rg * 8 + hh) * kD + dd) = make_float2(acc[hh][0], acc[hh][1]);
     }
     __syncthreads();
-    float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
     for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
       const int hh = idx >> 7, dd = idx & (kD - 1);
       float v = 0.f;
 #pragma unroll
       for (int rg = 0; rg < 8; ++rg) v += red[(rg * 8 + hh) * kD + dd];
-      out_head[idx] = v;
+      out_head[idx] = fmaf(s.wm[0][hh], v, window_o(hh, dd));
     }
   }
 }
@@ -1108,8 +1359,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }  // namespace
 
 cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, const void* q,
-                          int q_dtype, float* out, const SeqMap& sm, cudaStream_t s) {
+                          int q_dtype, float* out, const SeqMap& sm, const Fp16Kv& kv,
+                          cudaStream_t s) {
   DecodeArgs a;
+  const bool konly = p->cfg.v_bits == 0;
   a.packed = packed;
   a.meta = p->d_meta;
   a.rotpack = p->d_rotpack;
@@ -1130,13 +1383,48 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.n_tiles = p->n_tiles;
   a.tile_bytes = (int)p->tile_bytes;
   a.kb = p->cfg.k_bits;
-  a.stride = (int)((kTPS * p->tile_bytes + 127) & ~size_t(127));
+  // a stage: kTPS tiles, then (K-only) their fp16 value rows, 16 KB per tile
+  const size_t salign = konly ? 1024 : 128;
+  a.voff = (int)((kTPS * p->tile_bytes + salign - 1) & ~(salign - 1));
+  a.stride = konly ? a.voff + kTPS * kTile * kD * 2 : a.voff;
+  a.v_loads = 1;
+  a.v16 = kv.v;
+  a.vs0 = kv.vs[0];
+  a.vs1 = kv.vs[1];
+  a.vs2 = kv.vs[2];
+  a.rk = kv.rk;
+  a.rv = kv.rv;
+  a.rs0 = kv.rs[0];
+  a.rs1 = kv.rs[1];
+  a.rs2 = kv.rs[2];
+  a.rlens = kv.rlens;
+  a.rlen = (int)kv.rlen;
+  CUtensorMap vmap;
+  memset(&vmap, 0, sizeof(vmap));
+  if (konly) {
+    // (64 dims, T tokens, 2 dim halves, Hkv, B): one copy per tile brings both
+    // halves; without it, a 4-D map and a copy per half give the same layout
+    const uint64_t dims5[5] = {64, (uint64_t)T, 2, (uint64_t)p->cfg.n_kv_heads,
+                               (uint64_t)p->cfg.batch};
+    const uint64_t st5[4] = {(uint64_t)kv.vs[2] * 2, 128, (uint64_t)kv.vs[1] * 2,
+                             (uint64_t)kv.vs[0] * 2};
+    const uint32_t box5[5] = {64, (uint32_t)kTile, 2, 1, 1};
+    if (!encode_fp16_map(&vmap, 5, kv.v, dims5, st5, box5, true)) {
+      const uint64_t dims4[4] = {(uint64_t)kD, (uint64_t)T, (uint64_t)p->cfg.n_kv_heads,
+                                 (uint64_t)p->cfg.batch};
+      const uint64_t st4[3] = {(uint64_t)kv.vs[2] * 2, (uint64_t)kv.vs[1] * 2,
+                               (uint64_t)kv.vs[0] * 2};
+      const uint32_t box4[4] = {64, (uint32_t)kTile, 1, 1};
+      if (!encode_fp16_map(&vmap, 4, kv.v, dims4, st4, box4, true)) return cudaErrorNotSupported;
+      a.v_loads = 2;
+    }
+  }
   int dev_smem = 0;
   cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
   if (dev_smem < kSmemBytes) return cudaErrorInvalidValue;
   // stage area: below the table region, after DecodeSmem (the dynamic window may
   // start up to 1 KB above shared address 0)
-  const int area = (int)kTabSharedAddr - (int)((1024 + sizeof(DecodeSmem) + 127) & ~size_t(127));
+  const int area = (int)kTabSharedAddr - (int)((1024 + sizeof(DecodeSmem) + salign - 1) & ~(salign - 1));
   if (area < kTailBytes || area < kPackArea + a.stride) return cudaErrorInvalidValue;
   const int ring = std::min(kMaxRing, area / a.stride);
   if (ring < 2) return cudaErrorInvalidValue;
@@ -1151,7 +1439,8 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   splits = (int)std::min<int64_t>(splits, std::max<int64_t>(1, tiles_T));
   splits = std::max(1, std::min(splits, kMaxSplits));
   a.static_per = tiles_T * kStaticEighths / 8 / splits;
-  const int64_t budget = kPrefetchBudget / ((int64_t)p->n_heads * splits * a.tile_bytes);
+  const int64_t tile_in = a.tile_bytes + (konly ? kTile * kD * 2 : 0);  // bytes read per tile
+  const int64_t budget = kPrefetchBudget / ((int64_t)p->n_heads * splits * tile_in);
   a.prefetch = (int)std::max<int64_t>(0, std::min<int64_t>(a.static_per, budget));
   cudaError_t e = cudaErrorInvalidValue;
   const dim3 grid((unsigned)p->n_heads, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));
@@ -1160,8 +1449,10 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   case VB:                                                                                   \
     e = cudaFuncSetAttribute(decode_kernel<VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              kSmemBytes);                                                     \
-    if (e == cudaSuccess) e = launch_pdl(decode_kernel<VB>, grid, block, kSmemBytes, s, a);   \
+    if (e == cudaSuccess)                                                                    \
+      e = launch_pdl(decode_kernel<VB>, grid, block, kSmemBytes, s, vmap, a);                 \
     break;
+    GTQ_LAUNCH_VB(0)
     GTQ_LAUNCH_VB(1) GTQ_LAUNCH_VB(2) GTQ_LAUNCH_VB(3) GTQ_LAUNCH_VB(4)
     GTQ_LAUNCH_VB(5) GTQ_LAUNCH_VB(6) GTQ_LAUNCH_VB(7) GTQ_LAUNCH_VB(8)
 #undef GTQ_LAUNCH_VB

@@ -1,6 +1,7 @@
 // Internal declarations of libgtq (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -21,10 +22,19 @@ constexpr int kMaxSplits = 256;         // context splits per head in decode
 constexpr int kPartialStride = 4 + kD;  // (m, l, -, -, o[128]) per (split, q head)
 constexpr int kMergeGroup = 16;          // splits merged together at the first merge level
 constexpr int kMaxMergeGroups = kMaxSplits / kMergeGroup;
-constexpr int kPartialSlots = kMaxSplits + kMaxMergeGroups;  // per head: level 1 + level 2
+constexpr int kWindowSlot = kMaxSplits + kMaxMergeGroups;    // the fp16 window's partial
+constexpr int kPartialSlots = kWindowSlot + 1;  // per head: level 1 + level 2 + window
+constexpr int kMaxWindow = 1024;                // fp16 window rows per head (at most)
 constexpr int kStatusOverflow = 1;      // status word bits
 constexpr int kStatusTimeout = 2;
 constexpr int kStatusLayout = 4;        // a kernel found its shared-memory layout unusable
+
+// Byte offsets inside a packed tile: key codes, value codes (1024 vb), value
+// norms (128, only when values are coded), key norms (128 per group).
+__host__ __device__ constexpr int value_norm_offset(int kb, int vb) { return 1024 * (kb + vb); }
+__host__ __device__ constexpr int key_norm_offset(int kb, int vb) {
+  return 1024 * (kb + vb) + (vb > 0 ? 128 : 0);
+}
 
 // First LUT / threshold entry of width w (1..8).
 __host__ __device__ inline int lut_base(int w) { return (1 << w) - 2; }
@@ -230,6 +240,24 @@ cudaError_t build_b_images(const float* rows, int count, size_t stride, uint8_t*
                            cudaStream_t s);
 size_t b_image_bytes();
 cudaError_t build_code_lut(const float* thr, uint8_t* blob, cudaStream_t s);
+// Encodes a tiled fp16 tensor map (zero fill outside the extents); false if the
+// driver entry point is missing or rejects the description.  strides: bytes of
+// dims 1..rank-1.
+bool encode_fp16_map(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box, bool swizzle128);
+
+// fp16 operands of a decode (gtq_fp16_kv, checked): values of a K-only plan
+// and the window of recent tokens; strides in elements
+struct Fp16Kv {
+  const __half* v = nullptr;
+  int64_t vs[4] = {0, 0, 0, 0};
+  const __half* rk = nullptr;
+  const __half* rv = nullptr;
+  int64_t rs[4] = {0, 0, 0, 0};
+  const int32_t* rlens = nullptr;
+  int64_t rlen = 0;
+};
 cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, const void* q,
-                          int q_dtype, float* out, const SeqMap& sm, cudaStream_t s);
+                          int q_dtype, float* out, const SeqMap& sm, const Fp16Kv& kv,
+                          cudaStream_t s);
 }  // namespace gtq

@@ -149,8 +149,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
   const HeadMeta& m = s.meta;
   const T* kbase = reinterpret_cast<const T*>(a.k) + b * a.s0 + h * a.s1;
   const T* vbase = reinterpret_cast<const T*>(a.v) + b * a.s0 + h * a.s1;
-  const int vcode_off = 1024 * a.kb, vnorm_off = 1024 * (a.kb + a.vb);
-  const int knorm_off = vnorm_off + 128;
+  const int vcode_off = 1024 * a.kb, vnorm_off = value_norm_offset(a.kb, a.vb);
+  const int knorm_off = key_norm_offset(a.kb, a.vb);
   const int64_t tile_first = t0 / kTile, tile_last = (t1 - 1) / kTile;
   const int tb = tid >> 4, rb = tid & 15;
   const float sqrt_d = sqrtf((float)kD);
@@ -222,6 +222,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quantize_kernel(QuantArgs a) {
     }
     __syncthreads();
     // ----------------------------------------------------------------- values
+    if (a.vb == 0) {  // K-only: the tile holds keys only
+      for (int i = tid; i < a.tile_bytes / 16; i += kQThreads)
+        reinterpret_cast<uint4*>(gimg)[i] = reinterpret_cast<const uint4*>(img)[i];
+      __syncthreads();
+      continue;
+    }
     load_tile<T>(s, vbase, tok0, t0, t1 - t0, a.s2);
     __syncthreads();
     if (tid < kTile) {

@@ -482,7 +482,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     // ----------------------------------------------------------- norm warps
     const int q = warp & 3, j = 32 * q + lane;  // token of the tile (= tensor-memory lane)
     const uint32_t trow = tmem + 256 + ((uint32_t)(32 * q) << 16);
-    const int norm_off = ROLE == 0 ? 1024 * (a.kb + a.vb) + 128 : 1024 * (a.kb + a.vb);
+    const int norm_off = ROLE == 0 ? key_norm_offset(a.kb, a.vb) : value_norm_offset(a.kb, a.vb);
     const int jj = j & 63, npos = 2 * ((jj & 7) * 8 + (jj >> 3));
     const int n_chunks = gi.n_chunks;
     int ovf = 0, it = 0;
@@ -823,6 +823,24 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
+bool encode_fp16_map(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box, bool swizzle128) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || rank < 1 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = (cuuint64_t)dims[i];
+    bx[i] = (cuuint32_t)box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = (cuuint64_t)strides[i];
+  }
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, st,
+             bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t build_b_images(const float* rows, int count, size_t stride, uint8_t* img,
                            cudaStream_t s) {
   b_image_kernel<<<count, 256, 0, s>>>(rows, stride, img);
@@ -845,6 +863,7 @@ cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, 
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap maps[2];
   const void* src[2] = {k, v};
+  if (p->cfg.v_bits == 0) src[1] = k;  // K-only: the value map is never used
   for (int r = 0; r < 2; ++r) {
     if (((uintptr_t)src[r] & 15) || ((st[0] * 2) & 15) || ((st[1] * 2) & 15) || ((st[2] * 2) & 15))
       return cudaErrorNotSupported;
@@ -891,6 +910,10 @@ cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, 
   const int share_v = per_head == 2 ? 1 : per_head - share_k;
   a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_k));
   a.ctas_v = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_v));
+  if (p->cfg.v_bits == 0) {  // K-only: every CTA of the head codes keys
+    a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, per_head));
+    a.ctas_v = 0;
+  }
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
   if (e != cudaSuccess) return e;

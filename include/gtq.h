@@ -93,7 +93,7 @@ typedef struct gtq_config {
   int32_t n_kv_heads;   /* Hkv >= 1; Hq / Hkv (the GQA group) must be 1..8      */
   int32_t head_dim;     /* d: 128 for quantize/decode; any even 4..128 for alloc*/
   int32_t k_bits;       /* key budget in bits per dim, 1..8                     */
-  int32_t v_bits;       /* value bits per dim, 1..8                             */
+  int32_t v_bits;       /* value bits per dim, 1..8; 0: K-only (fp16 values)    */
   int32_t max_bits;     /* widest block width, 1..8 (normally 8)                */
   int32_t rope_pairing; /* GTQ_PAIRING_*                                        */
   int32_t in_dtype;     /* GTQ_DTYPE_* of K and V                               */
@@ -136,7 +136,8 @@ GTQ_API int gtq_alloc_bits_from_energy(const gtq_config* cfg, const double* host
  * (uniform v_bits) of tokens [t0, t0 + n_tokens) into the packed cache.
  *   k_dev, v_dev  post-RoPE K and V, in_dtype, laid out like gtq_alloc_bits'
  *                 k_dev with the same 4 strides (strides[3] == 1); token t of
- *                 the cache is row t of these tensors.
+ *                 the cache is row t of these tensors.  A K-only plan
+ *                 (v_bits 0) codes keys alone and takes v_dev = NULL.
  *   packed_dev    the packed cache, >= gtq_packed_bytes(plan) bytes, 16-byte
  *                 aligned, caller-owned.  Tokens outside [t0, t0+n) keep their
  *                 bytes (appending to an existing cache is allowed).
@@ -167,6 +168,7 @@ GTQ_API int gtq_quantize_pack(gtq_plan* plan, const void* k_dev, const void* v_d
  */
 GTQ_API int gtq_decode_attn(gtq_plan* plan, const void* packed_dev, int64_t T,
                     const void* q_dev, int32_t q_dtype, float* out_dev, void* stream);
+/* (A K-only plan, v_bits 0, decodes through gtq_decode_attn_full below.) */
 
 /* ---- batches of sequences of their own lengths; paged caches ------------ */
 
@@ -218,10 +220,59 @@ GTQ_API int gtq_quantize_pack_ex(gtq_plan* plan, const void* k_dev, const void* 
 
 /* gtq_decode_attn over a layout: sequence b attends to its first len_b tokens
  * (T is an upper bound, <= t_capacity, that sizes the launch; a sequence of
- * length 0 gets a zero output).  lay may be NULL.  Errors as gtq_decode_attn. */
+ * length 0 gets a zero output).  lay may be NULL.  Errors as gtq_decode_attn;
+ * a K-only plan needs gtq_decode_attn_full (INVALID here). */
 GTQ_API int gtq_decode_attn_ex(gtq_plan* plan, const void* packed_dev, int64_t T,
                                const gtq_seq_layout* lay, const void* q_dev, int32_t q_dtype,
                                float* out_dev, void* stream);
+
+/*
+ * fp16 operands of a decode.
+ *
+ * K-only mode: a plan made with v_bits = 0 codes only the keys (the page's
+ * K-only quantization, Abstract); the values stay in fp16 in the caller's own
+ * cache and v_dev names them:
+ *   v_dev           fp16, element (b, h, t, i) at v_dev + b*v_strides[0] +
+ *                   h*v_strides[1] + t*v_strides[2] + i (v_strides[3] must be
+ *                   1; the others multiples of 8; v_dev 16-byte aligned).
+ *                   Rows t < the call's T are read (row t of sequence b only
+ *                   below len_b, as the keys), whatever layout the packed keys
+ *                   use.  NULL for plans with coded values.
+ * Recent window: the fp16 recent-key buffer the page's headline result does
+ * without (Abstract) -- the last tokens of a sequence kept in fp16 beside the
+ * packed cache.  The query attends to the packed tokens and the window rows in
+ * one softmax; window logits are q.k / sqrt(d) on the fp16 keys, window
+ * values the fp16 values (original basis).
+ *   recent_k_dev, recent_v_dev  fp16 post-RoPE keys and values, element
+ *                   (b, h, r, i) at base + b*recent_strides[0] +
+ *                   h*recent_strides[1] + r*recent_strides[2] + i
+ *                   (recent_strides[3] must be 1, the others multiples of 4;
+ *                   bases 8-byte aligned).
+ *   recent_lens_dev device int32 [batch]: window rows of sequence b (clamped
+ *                   to [0, recent_len]), or NULL: recent_len for every one.
+ *   recent_len      rows per head, 0..1024; 0 = no window (the pointers may
+ *                   then be NULL).
+ * The window is attended by one CTA per KV head on the CUDA cores: its cost
+ * grows with recent_len (a few microseconds per layer at 128 rows).
+ */
+typedef struct gtq_fp16_kv {
+  const void* v_dev;
+  int64_t v_strides[4];
+  const void* recent_k_dev;
+  const void* recent_v_dev;
+  int64_t recent_strides[4];
+  const int32_t* recent_lens_dev;
+  int64_t recent_len;
+} gtq_fp16_kv;
+
+/* gtq_decode_attn_ex with fp16 operands (kv may be NULL: none).  A K-only plan
+ * requires kv->v_dev, a plan with coded values forbids it.  A sequence whose
+ * packed part and window are both empty gets a zero output.
+ * Errors as gtq_decode_attn; INVALID also for a bad kv. */
+GTQ_API int gtq_decode_attn_full(gtq_plan* plan, const void* packed_dev, int64_t T,
+                                 const gtq_seq_layout* lay, const gtq_fp16_kv* kv,
+                                 const void* q_dev, int32_t q_dtype, float* out_dev,
+                                 void* stream);
 
 /* gtq_free -- release the plan and its device memory.  Synchronises the plan's
  * device (cudaFree).  NULL is accepted.  Returns GTQ_OK or GTQ_ERR_CUDA. */
@@ -325,7 +376,8 @@ GTQ_API int gtq_rotation(uint64_t seed, int32_t tag, int32_t m, double* out);
  *                              16 i + g + 8 (x>>1 & 1), token
  *                              16 (x>>3) + 2c + (x & 1) + 8 (x>>2 & 1), at bits
  *                              [x v_bits, (x+1) v_bits).  Dim = row of R_V.
- *   next 128 bytes             value norms, fp16 [g][u] -> token g + 8u.
+ *   next 128 bytes             value norms, fp16 [g][u] -> token g + 8u
+ *                              (absent, like the value codes, when v_bits = 0).
  *   next 128 * 8 bytes         key norms, fp16 [group][g][u] (groups in the
  *                              descending-width order; unused groups unwritten).
  */

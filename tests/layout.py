@@ -20,7 +20,12 @@ TILE = 64
 
 
 def tile_bytes(kb: int, vb: int) -> int:
-    return 1024 * (kb + vb) + 128 + 128 * 8
+    """vb = 0: keys only (no value codes and no value norms)."""
+    return 1024 * (kb + vb) + (128 if vb else 0) + 128 * 8
+
+
+def _knorm(kb: int, vb: int) -> int:
+    return 1024 * (kb + vb) + (128 if vb else 0)
 
 
 def layout_groups(bits) -> list:
@@ -95,10 +100,12 @@ def read_head(buf: np.ndarray, bits, kb: int, vb: int, T: int):
     for gi, (w, st, jj, rr) in _key_maps(bits).items():
         codes = np.zeros((n * TILE, groups[gi][1]), np.int64)
         codes[(tok + jj[None, :]).ravel(), np.tile(rr, n)] = _gather(kbits, st, w).ravel()
-        nm = tiles[:, 1024 * (kb + vb) + 128 + gi * 128:][:, :128].copy().view(np.float16)
+        nm = tiles[:, _knorm(kb, vb) + gi * 128:][:, :128].copy().view(np.float16)
         n16 = np.zeros(n * TILE, np.float16)
         n16[(tok + _norm_map()[None, :]).ravel()] = nm.ravel()
         keys.append((w, codes[:T], n16[:T]))
+    if vb == 0:
+        return keys, None, None
     st, jj, dd = _value_map(vb)
     vcodes = np.zeros((n * TILE, 128), np.int64)
     vcodes[(tok + jj[None, :]).ravel(), np.tile(dd, n)] = _gather(vbits, st, vb).ravel()
@@ -113,7 +120,7 @@ def write_head(bits, key_groups: list, vcodes: np.ndarray, vnorm16: np.ndarray, 
     """Inverse of read_head (tokens >= T of the last tile are zero).
     key_groups: list of (width, codes [T, m], norm16 [T]) in descending width."""
     tb = tile_bytes(kb, vb)
-    T = vcodes.shape[0]
+    T = (vcodes.shape[0] if vcodes is not None else np.asarray(key_groups[0][1]).shape[0])
     n = (T + TILE - 1) // TILE
     assert [w for (w, _) in layout_groups(bits)] == [g[0] for g in key_groups]
     pad = n * TILE - T
@@ -127,20 +134,22 @@ def write_head(bits, key_groups: list, vcodes: np.ndarray, vnorm16: np.ndarray, 
         codes = padrows(np.asarray(key_groups[gi][1], np.int64))
         vals = codes[(tok + jj[None, :]), rr[None, :]]
         _scatter(kbits, st, vals, w)
-    st, jj, dd = _value_map(vb)
-    vbits = np.zeros((n, 1024 * vb * 8), np.uint8)
-    vc = padrows(np.asarray(vcodes, np.int64))
-    _scatter(vbits, st, vc[(tok + jj[None, :]), dd[None, :]], vb)
     out = np.zeros((n_tiles, tb), np.uint8)
     out[:n, :1024 * kb] = np.packbits(kbits, axis=1, bitorder="little")
-    out[:n, 1024 * kb:1024 * (kb + vb)] = np.packbits(vbits, axis=1, bitorder="little")
     nmap = _norm_map()
-    vn = padrows(np.asarray(vnorm16, np.float16))[(tok + nmap[None, :])]
-    o = 1024 * (kb + vb)
-    out[:n, o:o + 128] = vn.view(np.uint8).reshape(n, 128)
+    if vb:
+        st, jj, dd = _value_map(vb)
+        vbits = np.zeros((n, 1024 * vb * 8), np.uint8)
+        vc = padrows(np.asarray(vcodes, np.int64))
+        _scatter(vbits, st, vc[(tok + jj[None, :]), dd[None, :]], vb)
+        out[:n, 1024 * kb:1024 * (kb + vb)] = np.packbits(vbits, axis=1, bitorder="little")
+        vn = padrows(np.asarray(vnorm16, np.float16))[(tok + nmap[None, :])]
+        o = 1024 * (kb + vb)
+        out[:n, o:o + 128] = vn.view(np.uint8).reshape(n, 128)
+    o = _knorm(kb, vb)
     for gi, (w, codes, n16) in enumerate(key_groups):
         kn = padrows(np.asarray(n16, np.float16))[(tok + nmap[None, :])]
-        out[:n, o + 128 + gi * 128:o + 256 + gi * 128] = kn.view(np.uint8).reshape(n, 128)
+        out[:n, o + gi * 128:o + 128 + gi * 128] = kn.view(np.uint8).reshape(n, 128)
     return out.ravel()
 
 
