@@ -63,10 +63,11 @@ constexpr uint32_t kTabSharedAddr = 163840;   // shared address of the lookup ta
 constexpr int kSmemBytes = (int)kTabSharedAddr + kDecodeImageBytes;
 constexpr int kPackPrefix = 24576;            // rotation-pack bytes fetched with the metadata
 constexpr int kPackArea = (int)((kRotPackBytes + 127) & ~size_t(127));
-constexpr int kWoBytes = kCWarps * 8 * kD * 4;           // warps' o at the merge
-constexpr int kScratchBytes = 2 * 8 * kPartialStride * 4;  // split-merge scratch
-constexpr int kRvOff = (kWoBytes + kScratchBytes + 127) & ~127;
-constexpr int kTailBytes = kRvOff + kD * kD * 4;          // + R_V
+constexpr int kWoStride = kD + 4;                          // floats per (warp, head) row
+constexpr int kWoBytes = kCWarps * 8 * kWoStride * 4;      // warps' o at the merge
+constexpr int kRvFragBytes = 8 * 8 * 32 * 32;             // R_V^T fragments (fp16 hi + lo)
+constexpr int kRvOff = (kWoBytes + 127) & ~127;
+constexpr int kTailBytes = kRvOff + kRvFragBytes;
 constexpr uint64_t kWaitNs = 2000000000ull;    // bound of one wait
 constexpr int64_t kPrefetchBudget = 48ll << 20;  // bytes of L2 prefetch per launch
 static_assert(kTabSharedAddr % kDecTabAlign == 0, "table region alignment");
@@ -77,7 +78,7 @@ struct DecodeArgs {
   const HeadMeta* meta;
   const float* rotpack;    // [heads][kRotPackMaxWords]
   const void* q;           // [B][Hq][128] fp16 or fp32 (q_fp32)
-  const float* rot_v;      // R_V [128][128]
+  const uint4* rv_frag;    // R_V^T as mma A fragments: [m-tile][k-tile][lane] {hi, lo}
   float* out;              // [B][Hq][128]
   const uint4* dec_image;  // lookup tables (kDecodeImageBytes)
   float* partials;         // [heads][kPartialSlots][8][kPartialStride]
@@ -243,8 +244,8 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
 struct DecodeSmem {
   alignas(16) HeadMeta meta;
   uint4 qf[kMaxKt][32];        // per k-tile & lane: hi(slot A), hi(slot B), lo(A), lo(B)
-  alignas(16) float qa[8][kD];  // queries, then q_rot (scaled), then the merged o_rot
-  alignas(16) float qb[8][kD];  // queries gathered in each group's coordinate order
+  alignas(16) float qa[8][kD];  // gathered queries [coordinate][head], then the merged o_rot
+  alignas(16) float qb[8][kD];  // the raw queries (bulk copy), then q_rot (scaled)
   uint4 gdesc[kMaxGroups];      // W | split << 4 | k16 tiles << 8 | half k-tile << 16; key
                                 // offset; first k-tile; -
   uint64_t tab_bar;             // lookup tables landed
@@ -469,69 +470,49 @@ __device__ bool arrive_last(unsigned* ticket, unsigned count, int* flag) {
 
 // Merge partials [first, first + count) (count <= kMergeGroup) of the 8 query
 // heads: M = max m_j, L = sum 2^(m_j - M) l_j, o = sum 2^(m_j - M) o_j.  Written
-// as a partial to dst (global) or, normalised (o / L), to o_rot (shared).
-// Work item = (query head, parity of j) per warp, lane = 4 dims: a warp reads
-// whole partial rows (coalesced), all of its up to 8 partials in flight at
-// once; the two parities combine through `scratch` (shared, 2 x 8 x
-// kPartialStride floats).  Partials come from other CTAs: loads bypass L1.
+// as a partial to dst (global) or, normalised (o / L), to o_rot (shared) with
+// (M, L) to hm / hl.  Warp hh (< 8) takes query head hh, lane = 4 dims: whole
+// partial rows (coalesced), every load in flight at once, one pass.  Partials
+// come from other CTAs: loads bypass L1.  The caller synchronises afterwards.
 __device__ __noinline__ void merge_partials(const float* head_parts, int first, int count,
-                                            float* dst, float (*o_rot)[kD], float* scratch,
-                                            float* hm, float* hl) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int item = warp; item < 16; item += nwarps) {
-    const int hh = item >> 1, sub = item & 1;
-    float2 ml[kMergeGroup / 2];
-    float4 oj[kMergeGroup / 2];
+                                            float* dst, float (*o_rot)[kD], float* hm, float* hl) {
+  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int hh = threadIdx.x >> 5; hh < 8; hh += nwarps) {
+    float2 ml[kMergeGroup];
+    float4 oj[kMergeGroup];
 #pragma unroll
-    for (int b = 0; b < kMergeGroup / 2; ++b) {
-      const int j = sub + 2 * b;
-      ml[b] = make_float2(-1e30f, 0.f);
-      oj[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < kMergeGroup; ++j) {
+      ml[j] = make_float2(-1e30f, 0.f);
+      oj[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < count) {
         const float* pj = head_parts + ((size_t)(first + j) * 8 + hh) * kPartialStride;
-        ml[b] = __ldcg(reinterpret_cast<const float2*>(pj));
-        oj[b] = __ldcg(reinterpret_cast<const float4*>(pj + 4) + lane);
+        ml[j] = __ldcg(reinterpret_cast<const float2*>(pj));
+        oj[j] = __ldcg(reinterpret_cast<const float4*>(pj + 4) + lane);
       }
     }
     float M = ml[0].x;
 #pragma unroll
-    for (int b = 1; b < kMergeGroup / 2; ++b) M = fmaxf(M, ml[b].x);
+    for (int j = 1; j < kMergeGroup; ++j) M = fmaxf(M, ml[j].x);
     float L = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int b = 0; b < kMergeGroup / 2; ++b) {
-      const float w = exp2f(ml[b].x - M);
-      L = fmaf(w, ml[b].y, L);
-      o.x = fmaf(w, oj[b].x, o.x);
-      o.y = fmaf(w, oj[b].y, o.y);
-      o.z = fmaf(w, oj[b].z, o.z);
-      o.w = fmaf(w, oj[b].w, o.w);
+    for (int j = 0; j < kMergeGroup; ++j) {
+      const float w = exp2f(ml[j].x - M);
+      L = fmaf(w, ml[j].y, L);
+      o.x = fmaf(w, oj[j].x, o.x);
+      o.y = fmaf(w, oj[j].y, o.y);
+      o.z = fmaf(w, oj[j].z, o.z);
+      o.w = fmaf(w, oj[j].w, o.w);
     }
-    float* sc = scratch + (size_t)(sub * 8 + hh) * kPartialStride;
-    reinterpret_cast<float4*>(sc + 4)[lane] = o;
-    if (lane == 0) *reinterpret_cast<float2*>(sc) = make_float2(M, L);
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < 8 * 32; idx += blockDim.x) {
-    const int hh = idx >> 5, d4 = idx & 31;
-    const float* s0 = scratch + (size_t)hh * kPartialStride;
-    const float* s1 = scratch + (size_t)(8 + hh) * kPartialStride;
-    const float2 ml0 = *reinterpret_cast<const float2*>(s0), ml1 = *reinterpret_cast<const float2*>(s1);
-    const float4 o0 = reinterpret_cast<const float4*>(s0 + 4)[d4];
-    const float4 o1 = reinterpret_cast<const float4*>(s1 + 4)[d4];
-    const float M = fmaxf(ml0.x, ml1.x), w0 = exp2f(ml0.x - M), w1 = exp2f(ml1.x - M);
-    const float L = w0 * ml0.y + w1 * ml1.y;
-    const float4 o = make_float4(w0 * o0.x + w1 * o1.x, w0 * o0.y + w1 * o1.y, w0 * o0.z + w1 * o1.z,
-                                 w0 * o0.w + w1 * o1.w);
     if (dst) {
       float* pd = dst + hh * kPartialStride;
-      reinterpret_cast<float4*>(pd + 4)[d4] = o;
-      if (d4 == 0) *reinterpret_cast<float2*>(pd) = make_float2(M, L);
+      reinterpret_cast<float4*>(pd + 4)[lane] = o;
+      if (lane == 0) *reinterpret_cast<float2*>(pd) = make_float2(M, L);
     } else {
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      *reinterpret_cast<float4*>(&o_rot[hh][4 * d4]) =
+      *reinterpret_cast<float4*>(&o_rot[hh][4 * lane]) =
           make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
-      if (d4 == 0) {  // (M, L) of the whole cache, for the window's combination
+      if (lane == 0) {  // (M, L) of the whole cache, for the window's combination
         hm[hh] = M;
         hl[hh] = L;
       }
@@ -625,8 +606,8 @@ __device__ __noinline__ void window_partial(const WindowArgs a, DecodeSmem& s, i
       }
 #pragma unroll
     for (int hh = 0; hh < 8; ++hh)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) wo[(warp * kD + 4 * lane + e) * 8 + hh] = o[hh][e];
+      *reinterpret_cast<float4*>(wo + (warp * 8 + hh) * kWoStride + 4 * lane) =
+          make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
   }
   __syncthreads();
   if (tid < 8) {
@@ -642,11 +623,18 @@ __device__ __noinline__ void window_partial(const WindowArgs a, DecodeSmem& s, i
     *reinterpret_cast<float2*>(dst + hh * kPartialStride) = make_float2(M, L);
   }
   __syncthreads();
-  for (int idx = tid; idx < 8 * kD; idx += blockDim.x) {
-    const int hh = idx & 7, d = idx >> 3;
-    float v = 0.f;
-    for (int w = 0; w < ncw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * kD + d) * 8 + hh], v);
-    dst[hh * kPartialStride + 4 + d] = v;
+  for (int idx = tid; idx < 8 * kD / 4; idx += blockDim.x) {
+    const int hh = idx >> 5, d4 = idx & 31;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < ncw; ++w) {
+      const float sc = s.wsc[w][hh];
+      const float4 x = *reinterpret_cast<const float4*>(wo + (w * 8 + hh) * kWoStride + 4 * d4);
+      v.x = fmaf(sc, x.x, v.x);
+      v.y = fmaf(sc, x.y, v.y);
+      v.z = fmaf(sc, x.z, v.z);
+      v.w = fmaf(sc, x.w, v.w);
+    }
+    *reinterpret_cast<float4*>(dst + hh * kPartialStride + 4 + 4 * d4) = v;
   }
 }
 
@@ -732,9 +720,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // queries, metadata and the cache may come from the previous grid
   if (tid == 0) {
-    mbar_expect_tx(&s.meta_bar, (unsigned)(sizeof(HeadMeta) + kPackPrefix));
+    // the metadata, the first part of the rotation pack and the KV head's gq
+    // queries (contiguous) land on one barrier; the queries go to qb as they are
+    const unsigned qbytes = (unsigned)(a.gq * kD * (a.q_fp32 ? 4 : 2));
+    mbar_expect_tx(&s.meta_bar, (unsigned)(sizeof(HeadMeta) + kPackPrefix) + qbytes);
     bulk_copy(&s.meta, a.meta + head, sizeof(HeadMeta), &s.meta_bar);
     bulk_copy(pack, a.rotpack + (size_t)head * kRotPackMaxWords, kPackPrefix, &s.meta_bar);
+    bulk_copy(&s.qb[0][0],
+              reinterpret_cast<const uint8_t*>(a.q) + ((size_t)b * a.hkv + h) * qbytes, qbytes,
+              &s.meta_bar);
   }
   const int64_t T = a.seq_lens ? min((int64_t)a.seq_lens[b], a.T) : a.T;
   const int64_t tiles_T = (max(T, (int64_t)0) + kTile - 1) / kTile;
@@ -878,17 +872,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nct = ncw * 32;
     const int g = lane >> 2, t = lane & 3;
     const int pair = warp >> 1, wh = warp & 1;
-    // queries of this KV head (zero past the group size)
-    for (int i = tid; i < 8 * kD; i += nct) {
-      const int hh = i >> 7, d = i & (kD - 1);
-      float v = 0.f;
-      if (hh < a.gq) {
-        const size_t qi = ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq + hh) * kD + d;
-        v = a.q_fp32 ? reinterpret_cast<const float*>(a.q)[qi]
-                     : __half2float(reinterpret_cast<const __half*>(a.q)[qi]);
-      }
-      s.qa[hh][d] = v;
-    }
     failed = !mbar_wait(&s.meta_bar, 0);
     const HeadMeta& m = s.meta;
     if (tid == 0) {
@@ -906,36 +889,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     failed = !mbar_wait(&s.pack_bar, 0) || failed;
-    consumers_sync(nct);  // queries stored
-    // gather: qb[hh][p] = q[hh][dim of group coordinate p - first(g)]
+    // gather, transposed: qT[p][hh] = q[hh][dim of group coordinate p] (zero past
+    // the group size and the slots); qT lives in qa, the raw queries in qb
+    float(*qT)[8] = reinterpret_cast<float(*)[8]>(&s.qa[0][0]);
     const uint8_t* coord_dim = reinterpret_cast<const uint8_t*>(pack);
     for (int i = tid; i < 8 * kD; i += nct) {
-      const int hh = i >> 7, p = i & (kD - 1);
-      s.qb[hh][p] = (p >> 1) < m.n_slots ? s.qa[hh][coord_dim[p] & (kD - 1)] : 0.f;
+      const int p = i >> 3, hh = i & 7;
+      float v = 0.f;
+      if (hh < a.gq && (p >> 1) < m.n_slots) {
+        const int d = (hh << 7) | (coord_dim[p] & (kD - 1));
+        v = a.q_fp32 ? (&s.qb[0][0])[d] : __half2float(reinterpret_cast<const __half*>(&s.qb[0][0])[d]);
+      }
+      qT[p][hh] = v;
     }
     consumers_sync(nct);
-    // q_rot[hh][pos] = sum_c R_g[r][c] qb[hh][first + c] * log2(e) / (sqrt(d) sqrt(m_g))
-    for (int task = tid; task < 4 * kD; task += nct) {
-      const int pos = task & (kD - 1), hq = task >> 7, slot = pos >> 1;
-      float acc0 = 0.f, acc1 = 0.f, sc = 0.f;
+    // q_rot[hh][pos] = sum_c R_g[r][c] qT[first + c][hh] * log2(e) / (sqrt(d) sqrt(m_g)),
+    // into qb: a task is one position and four heads
+    for (int task = tid; task < 2 * kD; task += nct) {
+      const int pos = task & (kD - 1), h4 = (task >> 7) * 4, slot = pos >> 1;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float sc = 0.f;
       if (slot < m.n_slots) {
         const int gi = m.slot_group[slot], mm = m.grp_m[gi];
         const int first = 2 * m.grp_first_slot[gi], r = pos - first;
         int off = kRotPackHeaderWords;
         for (int gg = 0; gg < gi; ++gg) off += (int)m.grp_m[gg] * m.grp_m[gg];
         const float* Rc = pack + off + r;
-        const float* qa0 = &s.qb[2 * hq][first];
-        const float* qa1 = &s.qb[2 * hq + 1][first];
+        const float4* qc = reinterpret_cast<const float4*>(&qT[first][h4]);
 #pragma unroll 4
         for (int c = 0; c < mm; ++c) {
           const float rv = Rc[c * mm];
-          acc0 = fmaf(rv, qa0[c], acc0);
-          acc1 = fmaf(rv, qa1[c], acc1);
+          const float4 qv = qc[2 * c];
+          acc.x = fmaf(rv, qv.x, acc.x);
+          acc.y = fmaf(rv, qv.y, acc.y);
+          acc.z = fmaf(rv, qv.z, acc.z);
+          acc.w = fmaf(rv, qv.w, acc.w);
         }
         sc = m.inv_sqrt_m[gi] * (1.4426950408889634f * 0.08838834764831845f);
       }
-      s.qa[2 * hq][pos] = acc0 * sc;
-      s.qa[2 * hq + 1][pos] = acc1 * sc;
+      s.qb[h4][pos] = acc.x * sc;
+      s.qb[h4 + 1][pos] = acc.y * sc;
+      s.qb[h4 + 2][pos] = acc.z * sc;
+      s.qb[h4 + 3][pos] = acc.w * sc;
     }
     consumers_sync(nct);
     if (tid == 0) mbar_arrive(&s.done_bar);  // the pack's stages may be filled now
@@ -956,7 +951,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sl = tt + 4 * hf;  // slot within the k-tile
         const bool in = sl < m.kt_nslots[kt];
         const int pos = 2 * (m.kt_first_slot[kt] + sl);
-        const float v0 = in ? s.qa[gg][pos] : 0.f, v1 = in ? s.qa[gg][pos + 1] : 0.f;
+        const float v0 = in ? s.qb[gg][pos] : 0.f, v1 = in ? s.qb[gg][pos + 1] : 0.f;
         const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
         outv[hf] = pack_half2(h0, h1);
         outv[2 + hf] = pack_half2(__float2half_rn(v0 - __half2float(h0)),
@@ -1170,54 +1165,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (cta_failed && tid == 0) atomicOr(a.status, kStatusTimeout);
 
   // ------------------------------------------------- merge the warps in the CTA
-  float* wo = reinterpret_cast<float*>(stages);                       // [warp][8][128]
-  float* mscratch = reinterpret_cast<float*>(stages + kWoBytes);      // merge scratch
-  float* rv = reinterpret_cast<float*>(stages + kRvOff);              // R_V [128][128]
-  if (!producer) {
-    const int g = lane >> 2, t = lane & 3;
-    if (g == 0) {
-      s.wm[warp][2 * t] = mrun[0];
-      s.wm[warp][2 * t + 1] = mrun[1];
-      s.wl[warp][2 * t] = lrun[0];
-      s.wl[warp][2 * t + 1] = lrun[1];
-    }
-    // [warp][dim][head]: a lane's two heads are adjacent (one 8-byte store), and
-    // a half-warp's stores cover all 32 banks once
-    float* o = wo + warp * 8 * kD;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      *reinterpret_cast<float2*>(o + (16 * i + g) * 8 + 2 * t) = make_float2(O[i][0], O[i][1]);
-      *reinterpret_cast<float2*>(o + (16 * i + g + 8) * 8 + 2 * t) = make_float2(O[i][2], O[i][3]);
-    }
+  // wo[warp][head][kWoStride]: each warp's o rescaled to the CTA's maximum (the
+  // padded head stride keeps a warp's fragment stores free of bank conflicts)
+  float* wo = reinterpret_cast<float*>(stages);
+  uint4* rvf = reinterpret_cast<uint4*>(stages + kRvOff);  // R_V^T as A fragments
+  if (!producer && (lane >> 2) == 0) {
+    const int t = lane & 3;
+    *reinterpret_cast<float2*>(&s.wm[warp][2 * t]) = make_float2(mrun[0], mrun[1]);
+    *reinterpret_cast<float2*>(&s.wl[warp][2 * t]) = make_float2(lrun[0], lrun[1]);
   }
   __syncthreads();
-  if (tid < 8) {  // per query head: max over the warps, their scales and the sum of l
-    const int hh = tid;
-    float M = -1e30f;
-    for (int w = 0; w < ncw; ++w) M = fmaxf(M, s.wm[w][hh]);
-    float L = 0.f;
+  if (!producer) {
+    const int g = lane >> 2, t = lane & 3;
+    float M0 = -1e30f, M1 = -1e30f;
     for (int w = 0; w < ncw; ++w) {
-      const float sc = exp2f(s.wm[w][hh] - M);
-      s.wsc[w][hh] = sc;
-      L = fmaf(sc, s.wl[w][hh], L);
+      const float2 mw = *reinterpret_cast<const float2*>(&s.wm[w][2 * t]);
+      M0 = fmaxf(M0, mw.x);
+      M1 = fmaxf(M1, mw.y);
     }
-    s.hm[hh] = M;
-    s.hl[hh] = L;
+    const float sc0 = exp2f(mrun[0] - M0), sc1 = exp2f(mrun[1] - M1);
+    float* o0 = wo + (warp * 8 + 2 * t) * kWoStride;  // head 2t; head 2t + 1 one row on
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      o0[16 * i + g] = O[i][0] * sc0;
+      o0[kWoStride + 16 * i + g] = O[i][1] * sc1;
+      o0[16 * i + g + 8] = O[i][2] * sc0;
+      o0[kWoStride + 16 * i + g + 8] = O[i][3] * sc1;
+    }
+    if (warp == 0 && g == 0) {  // the CTA's (M, L) of heads 2t, 2t + 1
+      float L0 = 0.f, L1 = 0.f;
+      for (int w = 0; w < ncw; ++w) {
+        const float2 mw = *reinterpret_cast<const float2*>(&s.wm[w][2 * t]);
+        const float2 lw = *reinterpret_cast<const float2*>(&s.wl[w][2 * t]);
+        L0 = fmaf(exp2f(mw.x - M0), lw.x, L0);
+        L1 = fmaf(exp2f(mw.y - M1), lw.y, L1);
+      }
+      s.hm[2 * t] = M0;
+      s.hm[2 * t + 1] = M1;
+      s.hl[2 * t] = L0;
+      s.hl[2 * t + 1] = L1;
+    }
   }
   __syncthreads();
   float* head_parts = a.partials + (size_t)head * kPartialSlots * 8 * kPartialStride;
   float* part = head_parts + (size_t)split * 8 * kPartialStride;
   // this CTA's (m, l, o_rot): the output itself with a single split, else its
-  // partial in global memory
-  for (int idx = tid; idx < 8 * kD; idx += blockDim.x) {
-    const int hh = idx & 7, d = idx >> 3;
-    float v = 0.f;
-    for (int w = 0; w < ncw; ++w) v = fmaf(s.wsc[w][hh], wo[(w * kD + d) * 8 + hh], v);
+  // partial in global memory; a task is 4 dims of one head
+  for (int idx = tid; idx < 8 * kD / 4; idx += blockDim.x) {
+    const int hh = idx >> 5, d4 = idx & 31;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w)
+      if (w < ncw) {
+        const float4 x = *reinterpret_cast<const float4*>(wo + (w * 8 + hh) * kWoStride + 4 * d4);
+        v.x += x.x;
+        v.y += x.y;
+        v.z += x.z;
+        v.w += x.w;
+      }
     if (nsplit == 1) {
-      s.qa[hh][d] = s.hl[hh] > 0.f ? v / s.hl[hh] : 0.f;
+      const float inv = s.hl[hh] > 0.f ? 1.f / s.hl[hh] : 0.f;
+      *reinterpret_cast<float4*>(&s.qa[hh][4 * d4]) = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
     } else {
-      part[hh * kPartialStride + 4 + d] = v;
-      if (d == 0) *reinterpret_cast<float2*>(part + hh * kPartialStride) = make_float2(s.hm[hh], s.hl[hh]);
+      *reinterpret_cast<float4*>(part + hh * kPartialStride + 4 + 4 * d4) = v;
+      if (d4 == 0) *reinterpret_cast<float2*>(part + hh * kPartialStride) = make_float2(s.hm[hh], s.hl[hh]);
     }
   }
   // split 0 also attends the fp16 window, before its arrival publishes it
@@ -1229,13 +1240,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---------------- merge of the splits, without waiting: the last CTA to
   // arrive in a group of kMergeGroup splits merges the group into a
   // second-level partial, and the last group to finish merges those.  A CTA
-  // that may finish fetches R_V while it merges (coded values only).
+  // that may finish fetches R_V^T while it merges (coded values only).
   auto fetch_rv = [&]() -> bool {
     if (VB == 0) return false;
     if (tid == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_expect_tx(&s.rv_bar, (unsigned)(kD * kD * sizeof(float)));
-      bulk_copy(rv, a.rot_v, kD * kD * sizeof(float), &s.rv_bar);
+      mbar_expect_tx(&s.rv_bar, (unsigned)kRvFragBytes);
+      bulk_copy(rvf, a.rv_frag, kRvFragBytes, &s.rv_bar);
     }
     return true;
   };
@@ -1250,14 +1261,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (arrive_last(&head_tickets[1 + grp], (unsigned)n1, &s.flag)) {
       rv_issued = fetch_rv();
       if (n_grp == 1) {
-        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qa, mscratch, s.hm, s.hl);
+        merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qa, s.hm, s.hl);
         finish = true;
       } else {
         merge_partials(head_parts, grp * kMergeGroup, n1,
                        head_parts + (size_t)(kMaxSplits + grp) * 8 * kPartialStride, nullptr,
-                       mscratch, s.hm, s.hl);
+                       s.hm, s.hl);
         if (arrive_last(&head_tickets[0], (unsigned)n_grp, &s.flag)) {
-          merge_partials(head_parts, kMaxSplits, n_grp, nullptr, s.qa, mscratch, s.hm, s.hl);
+          merge_partials(head_parts, kMaxSplits, n_grp, nullptr, s.qa, s.hm, s.hl);
           finish = true;
         }
       }
@@ -1288,54 +1299,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     s.wm[0][tid] = cr;
     s.wl[0][tid] = cw;
   }
+  __syncthreads();
   float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
   auto window_o = [&](int hh, int dd) -> float {
     return a.rlen > 0 ? s.wl[0][hh] * __ldcg(wpart + hh * kPartialStride + 4 + dd) : 0.f;
   };
   if (VB == 0) {  // fp16 values: o_cache is already in the original basis
-    __syncthreads();
     for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
       const int hh = idx >> 7, dd = idx & (kD - 1);
       out_head[idx] = fmaf(s.wm[0][hh], s.qa[hh][dd], window_o(hh, dd));
     }
     return;
   }
-  // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r]: thread = (dd pair, 16 rows r of
-  // one r-group); o_rot^T in qb so that a warp reads its 8 heads of row r as two
-  // broadcasts; the 8 r-groups' partial sums are added through shared memory
-  {
-    float(*oT)[8] = reinterpret_cast<float(*)[8]>(&s.qb[0][0]);  // [r][head]
-    for (int i = tid; i < 8 * kD; i += blockDim.x) oT[i >> 3][i & 7] = s.qa[i & 7][i >> 3];
-    __syncthreads();
-    float* red = wo;  // [r-group][head][dim]
-    for (int task = tid; task < 512; task += blockDim.x) {
-      const int dd = 2 * (task & 63), rg = task >> 6;
-      float acc[8][2];
+  // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r] on the tensor cores: m-tile mt
+  // (dims [16 mt, 16 mt + 16)) goes to warp mt mod warps, A = R_V^T (fp16 hi + lo fragments), B =
+  // o_rot^T split into fp16 hi + lo; A_hi B_hi + A_hi B_lo + A_lo B_hi
+  for (int mt = warp; mt < 8; mt += blockDim.x >> 5) {
+    const int g = lane >> 2, t = lane & 3;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int hh = 0; hh < 8; ++hh) acc[hh][0] = acc[hh][1] = 0.f;
-#pragma unroll 4
-      for (int r = 16 * rg; r < 16 * rg + 16; ++r) {
-        const float2 w = *reinterpret_cast<const float2*>(rv + r * kD + dd);
-        const float4 oa = *reinterpret_cast<const float4*>(&oT[r][0]);
-        const float4 ob = *reinterpret_cast<const float4*>(&oT[r][4]);
-        const float ov[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          acc[hh][0] = fmaf(w.x, ov[hh], acc[hh][0]);
-          acc[hh][1] = fmaf(w.y, ov[hh], acc[hh][1]);
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < 8; ++hh)
-        *reinterpret_cast<float2*>(red + (rg * 8 + hh) * kD + dd) = make_float2(acc[hh][0], acc[hh][1]);
+    for (int kt = 0; kt < 8; ++kt) {
+      const uint4 fh = rvf[((mt * 8 + kt) * 32 + lane) * 2], fl = rvf[((mt * 8 + kt) * 32 + lane) * 2 + 1];
+      const uint32_t ah[4] = {fh.x, fh.y, fh.z, fh.w}, al[4] = {fl.x, fl.y, fl.z, fl.w};
+      const int r0 = 16 * kt + 2 * t;
+      const float2 x0 = *reinterpret_cast<const float2*>(&s.qa[g][r0]);
+      const float2 x1 = *reinterpret_cast<const float2*>(&s.qa[g][r0 + 8]);
+      const __half h00 = __float2half_rn(x0.x), h01 = __float2half_rn(x0.y);
+      const __half h10 = __float2half_rn(x1.x), h11 = __float2half_rn(x1.y);
+      const uint32_t bh0 = pack_half2(h00, h01), bh1 = pack_half2(h10, h11);
+      const uint32_t bl0 = pack_half2(__float2half_rn(x0.x - __half2float(h00)),
+                                      __float2half_rn(x0.y - __half2float(h01)));
+      const uint32_t bl1 = pack_half2(__float2half_rn(x1.x - __half2float(h10)),
+                                      __float2half_rn(x1.y - __half2float(h11)));
+      mma16816(c, ah, bh0, bh1);
+      mma16816(c, ah, bl0, bl1);
+      mma16816(c, al, bh0, bh1);
     }
-    __syncthreads();
-    for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
-      const int hh = idx >> 7, dd = idx & (kD - 1);
-      float v = 0.f;
+    // c[0], c[1]: dim 16 mt + g, heads 2t, 2t + 1; c[2], c[3]: dim + 8
+    const int dd = 16 * mt + g;
 #pragma unroll
-      for (int rg = 0; rg < 8; ++rg) v += red[(rg * 8 + hh) * kD + dd];
-      out_head[idx] = fmaf(s.wm[0][hh], v, window_o(hh, dd));
+    for (int r = 0; r < 4; ++r) {
+      const int hh = 2 * t + (r & 1), d = dd + 8 * (r >> 1);
+      if (hh < a.gq) out_head[hh * kD + d] = fmaf(s.wm[0][hh], c[r], window_o(hh, d));
     }
   }
 }
@@ -1368,7 +1373,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.rotpack = p->d_rotpack;
   a.q = q;
   a.q_fp32 = q_dtype == GTQ_DTYPE_FP32;
-  a.rot_v = p->tab.rot_v;
+  a.rv_frag = reinterpret_cast<const uint4*>(p->tab.rv_frag);
   a.out = out;
   a.tickets = p->d_tickets;
   a.hkv = p->cfg.n_kv_heads;

@@ -170,6 +170,8 @@ struct Tables {
   double* rot_k;     // R_m for m = 2, 4, ..., 128, row-major, concatenated (fp64)
   float* rot_v;      // R_V 128 x 128 row-major (fp32)
   float* rot_vt;     // R_V^T (fp32): element [d][r] = R_V[r][d]
+  uint32_t* rv_frag; // R_V^T as m16n8k16 A fragments, fp16 hi then lo (64 KB):
+                     // word ((m * 8 + k) * 32 + lane) * 8 + {0..3 hi, 4..7 lo}
   double* dist;      // D(0..8)
   float* thr;        // fp32 thresholds, width w at thr_base(w)
   uint4* dec_image;  // kDecodeImageBytes: the decode kernel's lookup tables

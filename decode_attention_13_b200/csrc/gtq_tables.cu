@@ -252,6 +252,32 @@ int tables_for(int device, uint64_t seed, Tables* out) {
       llo[lut_base(w) + k] = __double2half(r.c[k] - (double)__half2float(h));
     }
   }
+  // R_V^T as the decode's A fragments: A[dd][r] = R_V[r][dd] for output dims dd
+  // (m-tile m: dd = 16 m + ...) and rotated coordinates r (k-tile k); register
+  // j of lane (g, t) holds row g + 8 (j & 1), columns 2t + 8 (j >> 1) and the
+  // next one (low half first), as fp16 hi and the fp16 remainder lo
+  std::vector<uint32_t> rvf((size_t)8 * 8 * 32 * 8);
+  for (int mt = 0; mt < 8; ++mt)
+    for (int kt = 0; kt < 8; ++kt)
+      for (int lane = 0; lane < 32; ++lane)
+        for (int j = 0; j < 4; ++j) {
+          const int dd = 16 * mt + (lane >> 2) + 8 * (j & 1);
+          const int r = 16 * kt + 2 * (lane & 3) + 8 * (j >> 1);
+          uint32_t wh = 0, wl = 0;
+          for (int e = 0; e < 2; ++e) {
+            const float v = rv[(size_t)(r + e) * kD + dd];
+            const __half hv = __float2half_rn(v);
+            const __half lv = __float2half_rn(v - __half2float(hv));
+            uint16_t uh, ul;
+            std::memcpy(&uh, &hv, 2);
+            std::memcpy(&ul, &lv, 2);
+            wh |= (uint32_t)uh << (16 * e);
+            wl |= (uint32_t)ul << (16 * e);
+          }
+          const size_t base = (((size_t)mt * 8 + kt) * 32 + lane) * 8;
+          rvf[base + j] = wh;
+          rvf[base + 4 + j] = wl;
+        }
   // decode lookup-table image (layout: gtq_internal.h, kTab*)
   std::vector<uint32_t> img(kDecodeImageBytes / 4, 0u);
   auto bits16 = [](__half h) { uint16_t u; std::memcpy(&u, &h, 2); return (uint32_t)u; };
@@ -287,6 +313,7 @@ int tables_for(int device, uint64_t seed, Tables* out) {
   cudaError_t e = up((void**)&t.rot_k, rk.data(), rk.size() * sizeof(double));
   if (e == cudaSuccess) e = up((void**)&t.rot_v, rv.data(), rv.size() * sizeof(float));
   if (e == cudaSuccess) e = up((void**)&t.rot_vt, rvt.data(), rvt.size() * sizeof(float));
+  if (e == cudaSuccess) e = up((void**)&t.rv_frag, rvf.data(), rvf.size() * sizeof(uint32_t));
   if (e == cudaSuccess) e = up((void**)&t.dist, dist.data(), dist.size() * sizeof(double));
   if (e == cudaSuccess) e = up((void**)&t.thr, thr.data(), thr.size() * sizeof(float));
   if (e == cudaSuccess) e = up((void**)&t.dec_image, img.data(), img.size() * sizeof(uint32_t));
