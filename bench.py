@@ -62,7 +62,10 @@ def peaks():
 
 def packed_bytes_per_token_head(kb, vb, g_k):
     """Algorithmic bytes one decode reads per (token, KV head): key codes,
-    group norms, value codes, value norm."""
+    group norms, value codes, value norm (K-only plans, vb = 0: the fp16 value
+    row of 256 bytes instead)."""
+    if vb == 0:
+        return 16 * kb + 2 * g_k + 2 * 128
     return 16 * kb + 2 * g_k + 16 * vb + 2
 
 
@@ -353,6 +356,37 @@ def time_graph(graph, steps, warmup, stream, barrier=lambda: None):
     return t0.elapsed_time(t1) / steps
 
 
+def mixed_length_line(cfgd, w, dev, stream, hbm, steps, seed=11):
+    """The batch's sequences at their own lengths (uniform in [T/4, T], int32
+    lengths on the device, gtq_decode_attn_ex): bytes = the tokens each
+    sequence holds."""
+    import numpy as np
+    import torch
+
+    import decode_attention_13_b200 as gtq
+
+    L, B, hkv, T = cfgd["layers"], cfgd["B"], cfgd["h_kv"], cfgd["T"]
+    kb, vb = cfgd["k_bits"], cfgd["v_bits"]
+    lens = np.random.default_rng(seed).integers(T // 4, T + 1, size=B).astype(np.int32)
+    lens_dev = torch.from_numpy(lens).to(dev)
+    lay = gtq.seq_layout(lens_dev)
+    per_tok = w["step_bytes"] / (L * B * hkv * T)  # mean packed bytes per (token, head)
+
+    def step():
+        for layer in range(L):
+            gtq.gtq_decode_attn_ex(w["plans"][layer], w["packed"][layer], T, w["qs"][layer],
+                                   w["outs"][layer], layout=lay, stream=stream)
+
+    g = _graph_of(step, stream)
+    ms = time_graph(g, steps, 3, stream)
+    nbytes = float(L * hkv * int(lens.sum())) * per_tok
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del g
+    return {"decode_ms_per_step": ms, "decode_gbs": gbs, "decode_frac": gbs / hbm,
+            "bytes_per_step": nbytes, "ctx_tokens_per_s": float(lens.sum()) / (ms * 1e-3),
+            "seq_lens": "uniform in [T/4, T], mean %.0f" % float(lens.mean())}
+
+
 def per_config_line(cfgd, rank, dev, stream, hbm, steps):
     """Decode and quantize-pack of one more workload, for the per_config block."""
     import torch
@@ -367,9 +401,128 @@ def per_config_line(cfgd, rank, dev, stream, hbm, steps):
            "bytes_per_step": w["step_bytes"], "quantize_pack_ms": q_ms,
            "quantize_pack_gbs": q_bytes / (q_ms * 1e-3) / 1e9,
            "quantize_pack_frac": q_bytes / (q_ms * 1e-3) / 1e9 / hbm, "timed_steps": steps}
-    del graph, w
+    del graph
+    if cfgd["B"] > 1:
+        out["mixed_lengths"] = mixed_length_line(cfgd, w, dev, stream, hbm, steps)
+    del w
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
+    return out
+
+
+def _graph_of(fn, stream):
+    import torch
+
+    for _ in range(2):
+        with torch.cuda.stream(stream):
+            fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    stream.synchronize()
+    return g
+
+
+def decode_variants(cfgd, w, dev, stream, hbm, steps, window=128, seed=7):
+    """The decode step of the same workload in the library's other modes, each
+    captured in a CUDA graph and timed like the headline: a paged pool (pages
+    in shuffled order, gtq_decode_attn_ex with a block table), K-only plans
+    (keys coded, values read in fp16, gtq_decode_attn_full) and an fp16 window
+    of recent tokens beside the packed cache."""
+    import numpy as np
+    import torch
+
+    import decode_attention_13_b200 as gtq
+
+    L, B, hq, hkv, T = cfgd["layers"], cfgd["B"], cfgd["h_q"], cfgd["h_kv"], cfgd["T"]
+    kb, vb = cfgd["k_bits"], cfgd["v_bits"]
+    out = {}
+
+    def line(ms, nbytes, **kw):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        d = {"decode_ms_per_step": ms, "decode_gbs": gbs, "decode_frac": gbs / hbm,
+             "bytes_per_step": nbytes, "timed_steps": steps}
+        d.update(kw)
+        return d
+
+    ref = [o.clone() for o in w["outs"]]
+    # ---- paged pool
+    tb = gtq.gtq_layout_tile_bytes(kb, vb)
+    n_tiles = (T + 63) // 64
+    rng = np.random.default_rng(seed)
+    pools, tables = [], []
+    for layer in range(L):
+        perm = torch.from_numpy(rng.permutation(B * n_tiles).astype(np.int64)).to(dev)
+        src = w["packed"][layer][:B * hkv * n_tiles * tb].view(B, hkv, n_tiles, tb)
+        pool = torch.empty(B * n_tiles * hkv * tb, dtype=torch.uint8, device=dev)
+        pool.view(B * n_tiles, hkv, tb)[perm] = src.permute(0, 2, 1, 3).reshape(B * n_tiles, hkv, tb)
+        pools.append(pool)
+        tables.append(perm.view(B, n_tiles).to(torch.int32).contiguous())
+    lays = [gtq.seq_layout(None, t) for t in tables]
+
+    def paged():
+        for layer in range(L):
+            gtq.gtq_decode_attn_ex(w["plans"][layer], pools[layer], T, w["qs"][layer],
+                                   w["outs"][layer], layout=lays[layer], stream=stream)
+
+    g = _graph_of(paged, stream)
+    ms = time_graph(g, steps, 3, stream)
+    diff = max(float((o - r).abs().max()) for o, r in zip(w["outs"], ref))
+    out["paged"] = line(ms, w["step_bytes"], max_abs_diff_vs_contiguous=diff,
+                        how="pages of one tile of every KV head, shuffled block table")
+    del g, pools, tables, lays
+    # ---- K-only plans (fp16 values)
+    plans, packed, g_k = [], [], []
+    for layer, (k, v) in enumerate(w["kv"]):
+        cfg = gtq.make_config(B, hq, hkv, kb, 0, T)
+        with torch.cuda.stream(stream):
+            p = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
+            buf = torch.empty(p.packed_bytes, dtype=torch.uint8, device=dev)
+            gtq.gtq_quantize_pack(p, k, None, 0, T, buf, stream=stream)
+        plans.append(p)
+        packed.append(buf)
+    stream.synchronize()
+    for p in plans:
+        bits = gtq.gtq_get_bits(p)
+        g_k.append([[len(set(int(x) for x in bits[b, h] if x > 0)) for h in range(hkv)]
+                    for b in range(B)])
+    kvs = [gtq.fp16_kv(v=v) for (_, v) in w["kv"]]
+
+    def konly():
+        for layer in range(L):
+            gtq.gtq_decode_attn_full(plans[layer], packed[layer], T, w["qs"][layer],
+                                     w["outs"][layer], kv=kvs[layer], stream=stream)
+
+    g = _graph_of(konly, stream)
+    ms = time_graph(g, steps, 3, stream)
+    nbytes = float(sum(T * packed_bytes_per_token_head(kb, 0, g_k[l][b][h])
+                       for l in range(L) for b in range(B) for h in range(hkv)))
+    out["key_only"] = line(ms, nbytes, k_bits=kb, v_bits=0,
+                           how="keys coded at k_bits, values read in fp16 from the caller's "
+                               "tensor (gtq_decode_attn_full)")
+    del g, plans, packed, kvs
+    # ---- fp16 window of recent tokens beside the packed cache
+    gen = torch.Generator(device=dev).manual_seed(seed)
+    rks = [torch.randn((B, hkv, window, 128), generator=gen, device=dev, dtype=torch.float16)
+           for _ in range(L)]
+    rvs = [torch.randn((B, hkv, window, 128), generator=gen, device=dev, dtype=torch.float16)
+           for _ in range(L)]
+    wkv = [gtq.fp16_kv(recent_k=a, recent_v=b) for a, b in zip(rks, rvs)]
+
+    def windowed():
+        for layer in range(L):
+            gtq.gtq_decode_attn_full(w["plans"][layer], w["packed"][layer], T, w["qs"][layer],
+                                     w["outs"][layer], kv=wkv[layer], stream=stream)
+
+    g = _graph_of(windowed, stream)
+    ms = time_graph(g, steps, 3, stream)
+    out["window"] = line(ms, w["step_bytes"] + float(L * B * hkv * window * 512),
+                         window_tokens=window,
+                         how="K%dV%d cache plus %d fp16 recent tokens per head in one softmax"
+                             % (kb, vb, window))
+    del g, rks, rvs, wkv
+    torch.cuda.synchronize()
     return out
 
 
@@ -527,7 +680,11 @@ def run_ours(args, rank, world):
     stream.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     ref_check = np.isfinite(out_host.numpy()).all()
-    del graph, w
+    del graph
+    variants = None
+    if rank == 0 and world == 1 and not args.no_extra and not args.seq_len:
+        variants = decode_variants(cfgd, w, dev, stream, hbm, min(args.steps, 400))
+    del w
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
 
@@ -601,6 +758,8 @@ def run_ours(args, rank, world):
         "outputs_finite": bool(ref_check),
     }
     res.update(extra)
+    if variants:
+        res["variants"] = variants
     if cpu:
         res["cpu_baseline"] = cpu
     if rank == 0:

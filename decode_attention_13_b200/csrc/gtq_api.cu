@@ -256,12 +256,12 @@ int gtq_decode_attn_full(gtq_plan* plan, const void* packed_dev, int64_t T,
   }
   if (kv && kv->recent_len != 0) {
     if (kv->recent_len < 0 || kv->recent_len > kMaxWindow) return GTQ_ERR_INVALID;
-    if (!kv->recent_k_dev || !kv->recent_v_dev || !aligned(kv->recent_k_dev, 8) ||
-        !aligned(kv->recent_v_dev, 8) || kv->recent_strides[3] != 1 ||
+    if (!kv->recent_k_dev || !kv->recent_v_dev || !aligned(kv->recent_k_dev, 16) ||
+        !aligned(kv->recent_v_dev, 16) || kv->recent_strides[3] != 1 ||
         !aligned(kv->recent_lens_dev, 4))
       return GTQ_ERR_INVALID;
     for (int i = 0; i < 3; ++i)
-      if (kv->recent_strides[i] < 0 || kv->recent_strides[i] % 4) return GTQ_ERR_INVALID;
+      if (kv->recent_strides[i] < 0 || kv->recent_strides[i] % 8) return GTQ_ERR_INVALID;
     f.rk = (const __half*)kv->recent_k_dev;
     f.rv = (const __half*)kv->recent_v_dev;
     for (int i = 0; i < 4; ++i) f.rs[i] = kv->recent_strides[i];

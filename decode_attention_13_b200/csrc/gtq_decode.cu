@@ -5,9 +5,9 @@
 // grid = (heads, splits), one CTA per SM, 2 * np consumer warps (np pairs) and
 // one producer warp:
 //   setup    before the grid-dependency wait: the constant lookup tables
-//            (bulk copy) and an L2 prefetch of the tiles this CTA is likely to
-//            get; after it: the head metadata, the key rotation blocks and the
-//            queries, then q_rot = M_h q for the 8 query heads of the KV head,
+//            (bulk copy; an L2 prefetch of the CTA's tiles there measured 8%
+//            slower over a 36-layer step); after it: the head metadata, the key
+//            rotation blocks and the queries, then q_rot = M_h q for the 8 query heads of the KV head,
 //            from each group's m x m block only, times log2(e) / (sqrt(d)
 //            sqrt(m_g)), and its fp16 hi / lo MMA fragments.
 //   loop     the producer takes tiles from a per-head counter (two at a time,
@@ -69,7 +69,6 @@ constexpr int kRvFragBytes = 8 * 8 * 32 * 32;             // R_V^T fragments (fp
 constexpr int kRvOff = (kWoBytes + 127) & ~127;
 constexpr int kTailBytes = kRvOff + kRvFragBytes;
 constexpr uint64_t kWaitNs = 2000000000ull;    // bound of one wait
-constexpr int64_t kPrefetchBudget = 48ll << 20;  // bytes of L2 prefetch per launch
 static_assert(kTabSharedAddr % kDecTabAlign == 0, "table region alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -96,14 +95,11 @@ struct DecodeArgs {
   int kb;
   int ring;           // stages
   int np;             // consumer warp pairs
-  int prefetch;       // tiles this CTA prefetches into L2 before the dependency wait
   int64_t static_per; // tiles [split * static_per, +static_per) are this CTA's; the rest
                       // (from splits * static_per on) go out through the tile counter
   // K-only plans
   int voff;           // bytes of a stage before its value rows (kTPS x 16 KB, swizzled)
   int v_loads;        // tensor copies per tile: 1 (5-D map) or 2 (4-D map, one per half)
-  const __half* v16;  // fp16 values (L2 prefetch only; the copies go through the map)
-  int64_t vs0, vs1, vs2;  // their strides in elements
   // fp16 window of recent tokens
   const __half* rk;
   const __half* rv;
@@ -169,11 +165,8 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr)
                : "memory");
 }
-__device__ __forceinline__ void prefetch_l2(const void* src, unsigned bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 // the packed cache is streamed once per call: evicted first, so that it does
-// not push the tables, metadata and the next layer's prefetched tiles out of L2
+// not push the tables and metadata out of L2
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -534,88 +527,199 @@ struct HeadView {
   }
 };
 
-// Partial (m, l, o) of the 8 query heads over the sequence's fp16 window rows,
-// with logits in base 2 like the cache's (log2(e) q.k / sqrt(d)).  The consumer
-// warps take rows in turn (lane = 4 dims, one online softmax per warp); the
-// warps then merge through shared memory and the result is written to dst in
-// the layout of a split's partial.  Every thread of the CTA calls it.
+// Window rows are attended in blocks of 32 by up to kWinWarps warps of each of
+// the first n_w splits; a block's K and V rows are staged in shared memory with
+// a padded row (conflict-free ldmatrix), then processed like a tile half of
+// the cache: scores by mma (K fp16 exact, q as fp16 hi + lo), online softmax
+// in base 2, P.V with A = V^T from a transposing ldmatrix, all in the original
+// basis.
+constexpr int kWinRowBytes = 2 * kD + 16;
+constexpr int kWinBufBytes = 2 * 32 * kWinRowBytes;  // K and V rows of one block
+constexpr int kWinWarps = 4;
+constexpr int kWinSplits = 16;                      // window partials per head (at most)
+constexpr int kWinBytes = kWinWarps * kWinBufBytes + kWinWarps * 8 * kWoStride * 4;
+static_assert(kWinBytes <= kTailBytes, "window staging fits in the merge area");
+static_assert(kWinSplits <= kMergeGroup, "window partials merge in one pass");
+
 struct WindowArgs {
   const void* q;
   const __half* rk;
   const __half* rv;
   int64_t rs0, rs1, rs2;
-  const int32_t* rlens;
-  int rlen, q_fp32, hkv, gq;
+  int q_fp32, hkv, gq;
 };
-__device__ __noinline__ void window_partial(const WindowArgs a, DecodeSmem& s, int b, int h,
-                                            int ncw, float* dst, float* wo) {
-  __syncthreads();  // wo and the warp scales are free
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t wl = a.rlens ? min(max((int64_t)a.rlens[b], (int64_t)0), (int64_t)a.rlen)
-                             : (int64_t)a.rlen;
-  if (warp < ncw) {
-    float qv[8][4], m[8], l[8], o[8][4];
-    const float qs = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+
+// Window rows of sequence b (clamped to [0, rlen]).
+__device__ __forceinline__ int64_t window_len(const int32_t* rlens, int rlen, int b) {
+  if (rlen <= 0) return 0;
+  return rlens ? min(max((int64_t)rlens[b], (int64_t)0), (int64_t)rlen) : (int64_t)rlen;
+}
+
+// This split's window blocks j = split + k n_w (32 rows each) -> partial
+// (m, l, o) of the 8 query heads at dst, in the layout of a split's partial.
+// Every thread of the CTA calls it; it uses the stage area, qf and the warp
+// tables, and leaves qa, hm and hl alone.
+__device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int b, int h,
+                                         int split, int n_w, int64_t wl, int ncw, uint8_t* area,
+                                         uint32_t area_sa, float* dst) {
+  __syncthreads();  // the stage area and the warp tables are free
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int nww = min(ncw, kWinWarps);
+  // B fragments of q in the original basis, times log2(e) / sqrt(d): fp16 hi, lo
+  const float qs = 1.4426950408889634f * 0.08838834764831845f;
+  for (int idx = tid; idx < 8 * 32; idx += blockDim.x) {
+    const int kt = idx >> 5, ln = idx & 31, gg = ln >> 2, tt = ln & 3;
+    uint32_t o4[4];
 #pragma unroll
-    for (int hh = 0; hh < 8; ++hh) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = 0.f;
-        if (hh < a.gq) {
-          const size_t qi = (((size_t)b * a.hkv + h) * a.gq + hh) * kD + 4 * lane + e;
-          v = a.q_fp32 ? reinterpret_cast<const float*>(a.q)[qi]
-                       : __half2float(reinterpret_cast<const __half*>(a.q)[qi]);
+    for (int hf = 0; hf < 2; ++hf) {
+      const int d = 16 * kt + 2 * tt + 8 * hf;
+      float v0 = 0.f, v1 = 0.f;
+      if (gg < a.gq) {
+        const size_t qi = (((size_t)b * a.hkv + h) * a.gq + gg) * kD + d;
+        if (a.q_fp32) {
+          v0 = reinterpret_cast<const float*>(a.q)[qi];
+          v1 = reinterpret_cast<const float*>(a.q)[qi + 1];
+        } else {
+          v0 = __half2float(reinterpret_cast<const __half*>(a.q)[qi]);
+          v1 = __half2float(reinterpret_cast<const __half*>(a.q)[qi + 1]);
         }
-        qv[hh][e] = v * qs;
-        o[hh][e] = 0.f;
       }
-      m[hh] = -1e30f;
-      l[hh] = 0.f;
+      v0 *= qs;
+      v1 *= qs;
+      const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
+      o4[hf] = pack_half2(h0, h1);
+      o4[2 + hf] = pack_half2(__float2half_rn(v0 - __half2float(h0)), __float2half_rn(v1 - __half2float(h1)));
     }
-    const __half* kr = a.rk + b * a.rs0 + h * a.rs1 + 4 * lane;
-    const __half* vr = a.rv + b * a.rs0 + h * a.rs1 + 4 * lane;
-    for (int64_t r = warp; r < wl; r += ncw) {
-      const uint2 kq = __ldg(reinterpret_cast<const uint2*>(kr + r * a.rs2));
-      const uint2 vq = __ldg(reinterpret_cast<const uint2*>(vr + r * a.rs2));
-      const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kq.x));
-      const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kq.y));
-      const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vq.x));
-      const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vq.y));
+    s.qf[kt][ln] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+  }
+  __syncthreads();
+  float* wo2 = reinterpret_cast<float*>(area + kWinWarps * kWinBufBytes);  // [warp][head][kWoStride]
+  if (warp < nww) {
+    uint8_t* kbuf = area + warp * kWinBufBytes;
+    uint8_t* vbuf = kbuf + 32 * kWinRowBytes;
+    const uint32_t ksa = area_sa + (uint32_t)(warp * kWinBufBytes), vsa = ksa + 32 * kWinRowBytes;
+    const __half* kr = a.rk + b * a.rs0 + h * a.rs1;
+    const __half* vr = a.rv + b * a.rs0 + h * a.rs1;
+    float mrun[2] = {-1e30f, -1e30f}, lrun[2] = {0.f, 0.f};
+    float O[8][4];
 #pragma unroll
-      for (int hh = 0; hh < 8; ++hh) {
-        float sc = qv[hh][0] * k01.x;
-        sc = fmaf(qv[hh][1], k01.y, sc);
-        sc = fmaf(qv[hh][2], k23.x, sc);
-        sc = fmaf(qv[hh][3], k23.y, sc);
-#pragma unroll
-        for (int x = 16; x >= 1; x >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, x);
-        const float mn = fmaxf(m[hh], sc), al = exp2f(m[hh] - mn), p = exp2f(sc - mn);
-        l[hh] = fmaf(l[hh], al, p);
-        o[hh][0] = fmaf(o[hh][0], al, p * v01.x);
-        o[hh][1] = fmaf(o[hh][1], al, p * v01.y);
-        o[hh][2] = fmaf(o[hh][2], al, p * v23.x);
-        o[hh][3] = fmaf(o[hh][3], al, p * v23.y);
-        m[hh] = mn;
+    for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
+    for (int k = warp;; k += nww) {
+      const int64_t r0 = 32 * ((int64_t)split + (int64_t)k * n_w);
+      if (r0 >= wl) break;
+      // rows r0 .. r0 + 31 (zero past the window's length)
+      for (int c = lane; c < 32 * 16; c += 32) {
+        const int row = c >> 4, col = c & 15;
+        uint4 kq = make_uint4(0u, 0u, 0u, 0u), vq = kq;
+        if (r0 + row < wl) {
+          kq = __ldg(reinterpret_cast<const uint4*>(kr + (r0 + row) * a.rs2 + 8 * col));
+          vq = __ldg(reinterpret_cast<const uint4*>(vr + (r0 + row) * a.rs2 + 8 * col));
+        }
+        *reinterpret_cast<uint4*>(kbuf + row * kWinRowBytes + 16 * col) = kq;
+        *reinterpret_cast<uint4*>(vbuf + row * kWinRowBytes + 16 * col) = vq;
       }
+      __syncwarp();
+      // scores: rows 16 mt + g (+ 8), heads 2t, 2t + 1; A = K rows (ldmatrix: matrix
+      // lane >> 3 holds rows + 8 (bit 0) and dims + 8 (bit 1))
+      float S_[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        S_[mt][0] = S_[mt][1] = S_[mt][2] = S_[mt][3] = 0.f;
+        const uint32_t arow = ksa + (uint32_t)((16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1)) * kWinRowBytes);
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt) {
+          uint32_t av[4];
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(av[0]), "=r"(av[1]), "=r"(av[2]), "=r"(av[3])
+                       : "r"(arow + (uint32_t)((2 * kt + (lane >> 4)) * 16))
+                       : "memory");
+          const uint4 qv = s.qf[kt][lane];
+          mma16816(S_[mt], av, qv.x, qv.y);
+          mma16816(S_[mt], av, qv.z, qv.w);
+        }
+      }
+      // online softmax over the block (rows past the window are -inf)
+      const bool full = r0 + 32 <= wl;
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int j = 16 * mt + g + 8 * (r >> 1);
+          if (!full && r0 + j >= wl) S_[mt][r] = -INFINITY;
+          mx[r & 1] = fmaxf(mx[r & 1], S_[mt][r]);
+        }
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], 4));
+        mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], 8));
+        mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], 16));
+      }
+      float alpha[2];
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const float mn = fmaxf(mrun[q2], mx[q2]);
+        alpha[q2] = exp2f(mrun[q2] - mn);
+        mrun[q2] = mn;
+        lrun[q2] *= alpha[q2];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        O[i][0] *= alpha[0];
+        O[i][2] *= alpha[0];
+        O[i][1] *= alpha[1];
+        O[i][3] *= alpha[1];
+      }
+      uint32_t PB[2][2];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        float pp[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          pp[r] = exp2f(S_[mt][r] - mrun[r & 1]);
+          lrun[r & 1] += pp[r];
+        }
+        PB[mt][0] = movmatrix_t(pack_half2(__float2half_rn(pp[0]), __float2half_rn(pp[1])));
+        PB[mt][1] = movmatrix_t(pack_half2(__float2half_rn(pp[2]), __float2half_rn(pp[3])));
+      }
+      // P.V: A = V^T (16 dims x 16 rows) by a transposing ldmatrix
+      const uint32_t vrow = vsa + (uint32_t)(((lane & 7) + 8 * (lane >> 4)) * kWinRowBytes);
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint32_t av[4];
+          ldmatrix_x4_trans(av, vrow + (uint32_t)(kk * 16 * kWinRowBytes + (2 * i + ((lane >> 3) & 1)) * 16));
+          mma16816(O[i], av, PB[kk][0], PB[kk][1]);
+        }
+      __syncwarp();  // the block's rows are read before the next block lands
     }
-    if (lane == 0)
 #pragma unroll
-      for (int hh = 0; hh < 8; ++hh) {
-        s.wm[warp][hh] = m[hh];
-        s.wl[warp][hh] = l[hh];
-      }
+    for (int hh = 0; hh < 2; ++hh) {
+      lrun[hh] += __shfl_xor_sync(0xffffffffu, lrun[hh], 4);
+      lrun[hh] += __shfl_xor_sync(0xffffffffu, lrun[hh], 8);
+      lrun[hh] += __shfl_xor_sync(0xffffffffu, lrun[hh], 16);
+    }
+    if (g == 0) {
+      *reinterpret_cast<float2*>(&s.wm[warp][2 * t]) = make_float2(mrun[0], mrun[1]);
+      *reinterpret_cast<float2*>(&s.wl[warp][2 * t]) = make_float2(lrun[0], lrun[1]);
+    }
+    float* o0 = wo2 + (warp * 8 + 2 * t) * kWoStride;
 #pragma unroll
-    for (int hh = 0; hh < 8; ++hh)
-      *reinterpret_cast<float4*>(wo + (warp * 8 + hh) * kWoStride + 4 * lane) =
-          make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+    for (int i = 0; i < 8; ++i) {
+      o0[16 * i + g] = O[i][0];
+      o0[kWoStride + 16 * i + g] = O[i][1];
+      o0[16 * i + g + 8] = O[i][2];
+      o0[kWoStride + 16 * i + g + 8] = O[i][3];
+    }
   }
   __syncthreads();
   if (tid < 8) {
     const int hh = tid;
     float M = -1e30f;
-    for (int w = 0; w < ncw; ++w) M = fmaxf(M, s.wm[w][hh]);
+    for (int w = 0; w < nww; ++w) M = fmaxf(M, s.wm[w][hh]);
     float L = 0.f;
-    for (int w = 0; w < ncw; ++w) {
+    for (int w = 0; w < nww; ++w) {
       const float sc = exp2f(s.wm[w][hh] - M);
       s.wsc[w][hh] = sc;
       L = fmaf(sc, s.wl[w][hh], L);
@@ -626,9 +730,9 @@ __device__ __noinline__ void window_partial(const WindowArgs a, DecodeSmem& s, i
   for (int idx = tid; idx < 8 * kD / 4; idx += blockDim.x) {
     const int hh = idx >> 5, d4 = idx & 31;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = 0; w < ncw; ++w) {
+    for (int w = 0; w < nww; ++w) {
       const float sc = s.wsc[w][hh];
-      const float4 x = *reinterpret_cast<const float4*>(wo + (w * 8 + hh) * kWoStride + 4 * d4);
+      const float4 x = *reinterpret_cast<const float4*>(wo2 + (w * 8 + hh) * kWoStride + 4 * d4);
       v.x = fmaf(sc, x.x, v.x);
       v.y = fmaf(sc, x.y, v.y);
       v.z = fmaf(sc, x.z, v.z);
@@ -686,35 +790,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the tables are the library's constants: safe to read before the wait
     mbar_expect_tx(&s.tab_bar, (unsigned)kDecodeImageBytes);
     bulk_copy(tab, a.dec_image, kDecodeImageBytes, &s.tab_bar);
-  }
-  // L2 prefetch of the first tiles of this CTA's static share.  A prefetch
-  // changes no value a later load returns, so it may run before the wait; the
-  // sizes read here may be stale, which only changes how much is prefetched.
-  // One prefetch covers the whole range: the copy engine's time goes by copies.
-  if (producer && lane == 0 && a.prefetch > 0 && !hv.pages) {
-    const int64_t Tp = a.seq_lens ? (int64_t)__ldcg(a.seq_lens + b) : a.T;
-    const int64_t tiles = (min(max(Tp, (int64_t)0), a.T) + kTile - 1) / kTile;
-    const int64_t t0 = (int64_t)split * a.static_per;
-    const int64_t n = min((int64_t)a.prefetch, tiles - t0);
-    const int64_t Tc = min(max(Tp, (int64_t)0), a.T);
-    // value rows [t0, t0 + n tiles) below the sequence's length, when contiguous
-    auto prefetch_values = [&](int64_t tt0, int64_t nt) {
-      if (VB > 0 || a.vs2 != kD) return;
-      const int64_t r0 = tt0 * kTile, r1 = min((tt0 + nt) * kTile, Tc);
-      if (r1 > r0)
-        prefetch_l2(a.v16 + b * a.vs0 + h * a.vs1 + r0 * kD, (unsigned)((r1 - r0) * kD * 2));
-    };
-    if (n > 0) {
-      prefetch_l2(hv.tile(a.packed, t0), (unsigned)(n * a.tile_bytes));
-      prefetch_values(t0, n);
-    }
-    const int64_t dyn0 = (int64_t)nsplit * a.static_per;
-    const int64_t dper = (tiles - dyn0 + nsplit - 1) / nsplit;
-    const int64_t d0 = dyn0 + (int64_t)split * dper, dn = min(dper, tiles - d0);
-    if (dper > 0 && dn > 0) {
-      prefetch_l2(hv.tile(a.packed, d0), (unsigned)(dn * a.tile_bytes));
-      prefetch_values(d0, dn);
-    }
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -1231,11 +1306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (d4 == 0) *reinterpret_cast<float2*>(part + hh * kPartialStride) = make_float2(s.hm[hh], s.hl[hh]);
     }
   }
-  // split 0 also attends the fp16 window, before its arrival publishes it
-  float* wpart = head_parts + (size_t)kWindowSlot * 8 * kPartialStride;
-  if (a.rlen > 0 && split == 0) {
-    const WindowArgs wa = {a.q, a.rk, a.rv, a.rs0, a.rs1, a.rs2, a.rlens, a.rlen, a.q_fp32, a.hkv, a.gq};
-    window_partial(wa, s, b, h, ncw, wpart, wo);
+  // the first n_w splits also attend the fp16 window's 32-row blocks, each
+  // into a window partial of its own, before their arrival publishes it
+  const int64_t wl = window_len(a.rlens, a.rlen, b);
+  const int n_w = (int)min((int64_t)min(nsplit, kWinSplits), (wl + 31) / 32);
+  if (split < n_w) {
+    const WindowArgs wa = {a.q, a.rk, a.rv, a.rs0, a.rs1, a.rs2, a.q_fp32, a.hkv, a.gq};
+    window_pass(wa, s, b, h, split, n_w, wl, ncw, stages, stage_sa,
+                head_parts + (size_t)(kWindowSlot + split) * 8 * kPartialStride);
   }
   // ---------------- merge of the splits, without waiting: the last CTA to
   // arrive in a group of kMergeGroup splits merges the group into a
@@ -1284,15 +1362,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) atomicOr(a.status, kStatusTimeout);
     return;
   }
-  // out = cr o_cache + cw o_window (o_cache normalised, o_window not): the
-  // two softmax parts rescaled to their common maximum
+  // the window's partials merged into qb (normalised) with (M_w, L_w) in wsc[0], [1]
+  if (n_w > 0) {
+    merge_partials(head_parts, kWindowSlot, n_w, nullptr, s.qb, s.wsc[0], s.wsc[1]);
+    __syncthreads();
+  }
+  // out = cr o_cache + cw o_window (both normalised): the two softmax parts
+  // weighted by their sums at their common maximum
   if (tid < 8) {
     float cr = 1.f, cw = 0.f;
-    if (a.rlen > 0) {
-      const float2 mlw = __ldcg(reinterpret_cast<const float2*>(wpart + tid * kPartialStride));
-      const float M = s.hm[tid], L = s.hl[tid], Mx = fmaxf(M, mlw.x);
-      const float wr = exp2f(M - Mx) * L, ww = exp2f(mlw.x - Mx);
-      const float den = fmaf(ww, mlw.y, wr);
+    if (n_w > 0) {
+      const float M = s.hm[tid], L = s.hl[tid], Mw = s.wsc[0][tid], Lw = s.wsc[1][tid];
+      const float Mx = fmaxf(M, Mw);
+      const float wr = exp2f(M - Mx) * L, ww = exp2f(Mw - Mx) * Lw;
+      const float den = wr + ww;
       cr = den > 0.f ? wr / den : 0.f;
       cw = den > 0.f ? ww / den : 0.f;
     }
@@ -1301,16 +1384,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
-  auto window_o = [&](int hh, int dd) -> float {
-    return a.rlen > 0 ? s.wl[0][hh] * __ldcg(wpart + hh * kPartialStride + 4 + dd) : 0.f;
-  };
-  if (VB == 0) {  // fp16 values: o_cache is already in the original basis
+  auto window_o = [&](int hh, int dd) -> float { return n_w > 0 ? s.wl[0][hh] * s.qb[hh][dd] : 0.f; };
+  if constexpr (VB == 0) {  // fp16 values: o_cache is already in the original basis
     for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
       const int hh = idx >> 7, dd = idx & (kD - 1);
       out_head[idx] = fmaf(s.wm[0][hh], s.qa[hh][dd], window_o(hh, dd));
     }
-    return;
-  }
+  } else {
   // out[hh][dd] = sum_r R_V[r][dd] o_rot[hh][r] on the tensor cores: m-tile mt
   // (dims [16 mt, 16 mt + 16)) goes to warp mt mod warps, A = R_V^T (fp16 hi + lo fragments), B =
   // o_rot^T split into fp16 hi + lo; A_hi B_hi + A_hi B_lo + A_lo B_hi
@@ -1342,6 +1422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hh = 2 * t + (r & 1), d = dd + 8 * (r >> 1);
       if (hh < a.gq) out_head[hh * kD + d] = fmaf(s.wm[0][hh], c[r], window_o(hh, d));
     }
+  }
   }
 }
 
@@ -1393,10 +1474,6 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.voff = (int)((kTPS * p->tile_bytes + salign - 1) & ~(salign - 1));
   a.stride = konly ? a.voff + kTPS * kTile * kD * 2 : a.voff;
   a.v_loads = 1;
-  a.v16 = kv.v;
-  a.vs0 = kv.vs[0];
-  a.vs1 = kv.vs[1];
-  a.vs2 = kv.vs[2];
   a.rk = kv.rk;
   a.rv = kv.rv;
   a.rs0 = kv.rs[0];
@@ -1444,9 +1521,6 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   splits = (int)std::min<int64_t>(splits, std::max<int64_t>(1, tiles_T));
   splits = std::max(1, std::min(splits, kMaxSplits));
   a.static_per = tiles_T * kStaticEighths / 8 / splits;
-  const int64_t tile_in = a.tile_bytes + (konly ? kTile * kD * 2 : 0);  // bytes read per tile
-  const int64_t budget = kPrefetchBudget / ((int64_t)p->n_heads * splits * tile_in);
-  a.prefetch = (int)std::max<int64_t>(0, std::min<int64_t>(a.static_per, budget));
   cudaError_t e = cudaErrorInvalidValue;
   const dim3 grid((unsigned)p->n_heads, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));
   switch (p->cfg.v_bits) {

@@ -22,8 +22,8 @@ constexpr int kMaxSplits = 256;         // context splits per head in decode
 constexpr int kPartialStride = 4 + kD;  // (m, l, -, -, o[128]) per (split, q head)
 constexpr int kMergeGroup = 16;          // splits merged together at the first merge level
 constexpr int kMaxMergeGroups = kMaxSplits / kMergeGroup;
-constexpr int kWindowSlot = kMaxSplits + kMaxMergeGroups;    // the fp16 window's partial
-constexpr int kPartialSlots = kWindowSlot + 1;  // per head: level 1 + level 2 + window
+constexpr int kWindowSlot = kMaxSplits + kMaxMergeGroups;    // the fp16 window's partials
+constexpr int kPartialSlots = kWindowSlot + 16;  // per head: level 1 + level 2 + window
 constexpr int kMaxWindow = 1024;                // fp16 window rows per head (at most)
 constexpr int kStatusOverflow = 1;      // status word bits
 constexpr int kStatusTimeout = 2;

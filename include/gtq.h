@@ -246,14 +246,14 @@ GTQ_API int gtq_decode_attn_ex(gtq_plan* plan, const void* packed_dev, int64_t T
  *   recent_k_dev, recent_v_dev  fp16 post-RoPE keys and values, element
  *                   (b, h, r, i) at base + b*recent_strides[0] +
  *                   h*recent_strides[1] + r*recent_strides[2] + i
- *                   (recent_strides[3] must be 1, the others multiples of 4;
- *                   bases 8-byte aligned).
+ *                   (recent_strides[3] must be 1, the others multiples of 8;
+ *                   bases 16-byte aligned).
  *   recent_lens_dev device int32 [batch]: window rows of sequence b (clamped
  *                   to [0, recent_len]), or NULL: recent_len for every one.
  *   recent_len      rows per head, 0..1024; 0 = no window (the pointers may
  *                   then be NULL).
- * The window is attended by one CTA per KV head on the CUDA cores: its cost
- * grows with recent_len (a few microseconds per layer at 128 rows).
+ * The window is attended on the tensor cores in blocks of 32 rows spread over
+ * up to 16 CTAs of each KV head, each of which writes a partial of its own.
  */
 typedef struct gtq_fp16_kv {
   const void* v_dev;
