@@ -91,7 +91,8 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
   alloc((void**)&p->d_rotpack, H * kRotPackBytes);
   if (cfg->head_dim == kD) alloc((void**)&p->d_bimg, H * b_image_bytes());
-  alloc((void**)&p->d_partials, H * kPartialSlots * 8 * kPartialStride * sizeof(float));
+  alloc((void**)&p->d_partials, H * (size_t)PartialSlots(decode_split_cap(p->n_sms, p->n_heads)).total *
+                                    8 * kPartialStride * sizeof(float));
   alloc((void**)&p->d_tickets, H * kTicketStride * sizeof(unsigned));
   alloc((void**)&p->d_status, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * kTicketStride * sizeof(unsigned));
@@ -315,7 +316,8 @@ size_t gtq_plan_device_bytes(const gtq_plan* plan) {
   const size_t H = plan->n_heads;
   size_t b = H * plan->n_blocks * sizeof(double) + H * plan->n_blocks + H * sizeof(HeadMeta) +
              H * kD * kD * sizeof(float) + H * kRotPackBytes +
-             H * kPartialSlots * 8 * kPartialStride * sizeof(float) +
+             H * (size_t)PartialSlots(decode_split_cap(plan->n_sms, plan->n_heads)).total * 8 *
+                 kPartialStride * sizeof(float) +
              H * kTicketStride * sizeof(unsigned) + sizeof(int);
   if (plan->cfg.head_dim == kD) b += H * b_image_bytes();
   return b;

@@ -80,7 +80,8 @@ struct DecodeArgs {
   const uint4* rv_frag;    // R_V^T as mma A fragments: [m-tile][k-tile][lane] {hi, lo}
   float* out;              // [B][Hq][128]
   const uint4* dec_image;  // lookup tables (kDecodeImageBytes)
-  float* partials;         // [heads][kPartialSlots][8][kPartialStride]
+  float* partials;         // [heads][slot_total][8][kPartialStride]
+  int slot_groups, slot_window, slot_total;  // PartialSlots of the plan
   unsigned* tickets;       // [heads][kTicketStride]
   int* status;
   const int32_t* seq_lens;     // [B] tokens per sequence, or null: all T
@@ -536,10 +537,9 @@ struct HeadView {
 constexpr int kWinRowBytes = 2 * kD + 16;
 constexpr int kWinBufBytes = 2 * 32 * kWinRowBytes;  // K and V rows of one block
 constexpr int kWinWarps = 4;
-constexpr int kWinSplits = 16;                      // window partials per head (at most)
 constexpr int kWinBytes = kWinWarps * kWinBufBytes + kWinWarps * 8 * kWoStride * 4;
 static_assert(kWinBytes <= kTailBytes, "window staging fits in the merge area");
-static_assert(kWinSplits <= kMergeGroup, "window partials merge in one pass");
+static_assert(kWindowPartials <= kMergeGroup, "window partials merge in one pass");
 
 struct WindowArgs {
   const void* q;
@@ -1282,7 +1282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
-  float* head_parts = a.partials + (size_t)head * kPartialSlots * 8 * kPartialStride;
+  float* head_parts = a.partials + (size_t)head * a.slot_total * 8 * kPartialStride;
   float* part = head_parts + (size_t)split * 8 * kPartialStride;
   // this CTA's (m, l, o_rot): the output itself with a single split, else its
   // partial in global memory; a task is 4 dims of one head
@@ -1309,11 +1309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the first n_w splits also attend the fp16 window's 32-row blocks, each
   // into a window partial of its own, before their arrival publishes it
   const int64_t wl = window_len(a.rlens, a.rlen, b);
-  const int n_w = (int)min((int64_t)min(nsplit, kWinSplits), (wl + 31) / 32);
+  const int n_w = (int)min((int64_t)min(nsplit, kWindowPartials), (wl + 31) / 32);
   if (split < n_w) {
     const WindowArgs wa = {a.q, a.rk, a.rv, a.rs0, a.rs1, a.rs2, a.q_fp32, a.hkv, a.gq};
     window_pass(wa, s, b, h, split, n_w, wl, ncw, stages, stage_sa,
-                head_parts + (size_t)(kWindowSlot + split) * 8 * kPartialStride);
+                head_parts + (size_t)(a.slot_window + split) * 8 * kPartialStride);
   }
   // ---------------- merge of the splits, without waiting: the last CTA to
   // arrive in a group of kMergeGroup splits merges the group into a
@@ -1343,10 +1343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         finish = true;
       } else {
         merge_partials(head_parts, grp * kMergeGroup, n1,
-                       head_parts + (size_t)(kMaxSplits + grp) * 8 * kPartialStride, nullptr,
+                       head_parts + (size_t)(a.slot_groups + grp) * 8 * kPartialStride, nullptr,
                        s.hm, s.hl);
         if (arrive_last(&head_tickets[0], (unsigned)n_grp, &s.flag)) {
-          merge_partials(head_parts, kMaxSplits, n_grp, nullptr, s.qa, s.hm, s.hl);
+          merge_partials(head_parts, a.slot_groups, n_grp, nullptr, s.qa, s.hm, s.hl);
           finish = true;
         }
       }
@@ -1364,7 +1364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // the window's partials merged into qb (normalised) with (M_w, L_w) in wsc[0], [1]
   if (n_w > 0) {
-    merge_partials(head_parts, kWindowSlot, n_w, nullptr, s.qb, s.wsc[0], s.wsc[1]);
+    merge_partials(head_parts, a.slot_window, n_w, nullptr, s.qb, s.wsc[0], s.wsc[1]);
     __syncthreads();
   }
   // out = cr o_cache + cw o_window (both normalised): the two softmax parts
@@ -1461,6 +1461,11 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.gq = p->g_q;
   a.dec_image = p->tab.dec_image;
   a.partials = p->d_partials;
+  const int split_cap = decode_split_cap(p->n_sms, p->n_heads);
+  const PartialSlots slots(split_cap);
+  a.slot_groups = slots.groups;
+  a.slot_window = slots.window;
+  a.slot_total = slots.total;
   a.status = p->d_status;
   a.seq_lens = sm.seq_lens;
   a.block_table = sm.table;
@@ -1516,10 +1521,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   const int64_t tiles_T = (T + kTile - 1) / kTile;
   // one CTA per SM; with many heads, round up so that late CTAs join heads that
   // still have tiles left (the counter balances the work within a head)
-  int splits = p->n_heads >= 16 ? (p->n_sms + p->n_heads - 1) / p->n_heads
-                                : std::max(1, p->n_sms / p->n_heads);
-  splits = (int)std::min<int64_t>(splits, std::max<int64_t>(1, tiles_T));
-  splits = std::max(1, std::min(splits, kMaxSplits));
+  int splits = (int)std::min<int64_t>(split_cap, std::max<int64_t>(1, tiles_T));
   a.static_per = tiles_T * kStaticEighths / 8 / splits;
   cudaError_t e = cudaErrorInvalidValue;
   const dim3 grid((unsigned)p->n_heads, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));

@@ -22,8 +22,23 @@ constexpr int kMaxSplits = 256;         // context splits per head in decode
 constexpr int kPartialStride = 4 + kD;  // (m, l, -, -, o[128]) per (split, q head)
 constexpr int kMergeGroup = 16;          // splits merged together at the first merge level
 constexpr int kMaxMergeGroups = kMaxSplits / kMergeGroup;
-constexpr int kWindowSlot = kMaxSplits + kMaxMergeGroups;    // the fp16 window's partials
-constexpr int kPartialSlots = kWindowSlot + 16;  // per head: level 1 + level 2 + window
+constexpr int kWindowPartials = 16;     // fp16 window partials per head (at most)
+
+// Context splits per head that a decode on n_heads heads may use (one CTA per
+// SM; with many heads rounded up, so that late CTAs join heads with tiles left).
+inline int decode_split_cap(int n_sms, int n_heads) {
+  const int s = n_heads >= 16 ? (n_sms + n_heads - 1) / n_heads : (n_sms / n_heads > 1 ? n_sms / n_heads : 1);
+  return s < kMaxSplits ? s : kMaxSplits;
+}
+// Partial slots of one head: the splits, then the first-level group merges,
+// then the window partials.
+struct PartialSlots {
+  int groups, window, total;
+  explicit PartialSlots(int split_cap)
+      : groups(split_cap),
+        window(split_cap + (split_cap + kMergeGroup - 1) / kMergeGroup),
+        total(window + kWindowPartials) {}
+};
 constexpr int kMaxWindow = 1024;                // fp16 window rows per head (at most)
 constexpr int kStatusOverflow = 1;      // status word bits
 constexpr int kStatusTimeout = 2;
@@ -206,7 +221,7 @@ struct gtq_plan {
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
   float* d_rotpack;   // [heads][kRotPackMaxWords] key rotation blocks for the decode kernel
   uint8_t* d_bimg;    // [heads] M_h as the quantizer's tensor-core B operand (64 KB each)
-  float* d_partials;  // [heads][kPartialSlots][8][kPartialStride]
+  float* d_partials;  // [heads][PartialSlots(decode_split_cap).total][8][kPartialStride]
   unsigned* d_tickets;  // [heads][kTicketStride] split-merge tickets and the tile counter
   int* d_status;      // device status word
 };
