@@ -282,6 +282,8 @@ def build_workload(cfgd, rank, dev, stream):
     for layer in range(L):
         k, v, q = synth.layer_torch(rank_seed(cfgd["index"], rank, layer), B, hkv, gq, T,
                                     theta=cfgd["theta"], decay=cfgd["decay"], device=dev)
+        # the inputs were drawn on torch's stream: the library's stream waits for them
+        stream.wait_stream(torch.cuda.current_stream(dev))
         cfg = gtq.make_config(B, hq, hkv, kb, vb, T)
         with torch.cuda.stream(stream):
             plan = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
@@ -306,8 +308,10 @@ def build_workload(cfgd, rank, dev, stream):
                                 for l in range(L) for b in range(B) for h in range(hkv)))
     # small caches: further copies, so that a timed loop reads cold data
     w["copies"] = cache_copies(w["step_bytes"])
-    w["packed_copies"] = [w["packed"]] + [[p.clone() for p in w["packed"]]
-                                          for _ in range(w["copies"] - 1)]
+    with torch.cuda.stream(stream):
+        w["packed_copies"] = [w["packed"]] + [[p.clone() for p in w["packed"]]
+                                              for _ in range(w["copies"] - 1)]
+    stream.synchronize()
     w["fp16_bytes"] = float(L * B * hkv * T * 2 * 128 * 2)
     return w
 
@@ -393,6 +397,7 @@ def mixed_length_line(cfgd, w, dev, stream, hbm, steps, seed=11):
     kb, vb = cfgd["k_bits"], cfgd["v_bits"]
     lens = np.random.default_rng(seed).integers(T // 4, T + 1, size=B).astype(np.int32)
     lens_dev = torch.from_numpy(lens).to(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
     lay = gtq.seq_layout(lens_dev)
     per_tok = w["step_bytes"] / (L * B * hkv * T)  # mean packed bytes per (token, head)
 
@@ -471,6 +476,7 @@ def decode_variants(cfgd, w, dev, stream, hbm, steps, window=128, seed=7):
         d.update(kw)
         return d
 
+    torch.cuda.current_stream(dev).wait_stream(stream)
     ref = [o.clone() for o in w["outs"]]
     # ---- paged pool
     tb = gtq.gtq_layout_tile_bytes(kb, vb)
@@ -484,6 +490,7 @@ def decode_variants(cfgd, w, dev, stream, hbm, steps, window=128, seed=7):
         pool.view(B * n_tiles, hkv, tb)[perm] = src.permute(0, 2, 1, 3).reshape(B * n_tiles, hkv, tb)
         pools.append(pool)
         tables.append(perm.view(B, n_tiles).to(torch.int32).contiguous())
+    stream.wait_stream(torch.cuda.current_stream(dev))  # pools and tables built on torch's stream
     lays = [gtq.seq_layout(None, t) for t in tables]
 
     def paged():
@@ -533,6 +540,7 @@ def decode_variants(cfgd, w, dev, stream, hbm, steps, window=128, seed=7):
            for _ in range(L)]
     rvs = [torch.randn((B, hkv, window, 128), generator=gen, device=dev, dtype=torch.float16)
            for _ in range(L)]
+    stream.wait_stream(torch.cuda.current_stream(dev))
     wkv = [gtq.fp16_kv(recent_k=a, recent_v=b) for a, b in zip(rks, rvs)]
 
     def windowed():
@@ -573,6 +581,7 @@ def memory_report(cfgd, rank, dev, stream, seq_lens=(131072, 262144, 524288)):
         for layer in range(L):
             k, v, q = synth.layer_torch((cfgd["index"], rank, layer), B, hkv, gq, T,
                                         theta=cfgd["theta"], decay=cfgd["decay"], device=dev)
+            stream.wait_stream(torch.cuda.current_stream(dev))
             cfg = gtq.make_config(B, hq, hkv, kb, vb, T)
             with torch.cuda.stream(stream):
                 plan = gtq.gtq_alloc_bits(cfg, k, T, stream=stream)
@@ -652,11 +661,12 @@ def run_ours(args, rank, world):
     # ---- the decode step, captured in a CUDA graph (only decode_kernel runs in it)
     graph, _ = decode_graph(cfgd, w, stream)
     clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    # warm-up after the sampler's start, so the timed steps begin at full clocks
     for i in range(max(3, args.warmup)):
         graph[i % len(graph)].replay()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
     copies = w["copies"]  # graphs over different copies of the cache, replayed in turn
     ms_local = time_graph(graph, args.steps, 0, stream, barrier)
     timed_steps = args.steps
