@@ -124,11 +124,10 @@ __global__ void __launch_bounds__(kAThreads) append_kernel(AppendArgs a) {
   const int head = blockIdx.x, role = blockIdx.y;
   const int b = head / a.hkv, h = head % a.hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // tokens of this sequence among the call's: [t0, t0 + n)
-  const int64_t len = a.sm.len(b, a.cap);
-  const int64_t t0 = a.sm.tail ? max((int64_t)0, len - a.n) : a.t0;
-  const int n = (int)max((int64_t)0, min((int64_t)a.n, len - t0));
-  if (n == 0) return;
+  // Before the grid-dependency wait only the plan's constants are read (its
+  // metadata, rotation blocks and thresholds, written when the plan was made);
+  // the lengths, the new rows and the packed cache may come from the previous
+  // grid and are read or written after it.
   if (tid == 0) {
     m = a.meta[head];
     ovf = 0;
@@ -152,6 +151,17 @@ __global__ void __launch_bounds__(kAThreads) append_kernel(AppendArgs a) {
         : "memory");
   }
   for (int i = tid; i < kThrEntries; i += kAThreads) thr[i] = a.thr[i];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // tokens of this sequence among the call's: [t0, t0 + n)
+  const int64_t len = a.sm.len(b, a.cap);
+  const int64_t t0 = a.sm.tail ? max((int64_t)0, len - a.n) : a.t0;
+  const int n = (int)max((int64_t)0, min((int64_t)a.n, len - t0));
+  if (n == 0) {  // nothing to write: only the rotation copy must land before the exit
+    __syncthreads();
+    if (tid == 0 && !wait_phase0(&bar)) atomicOr(a.status, kStatusTimeout);
+    return;
+  }
   const T* src = reinterpret_cast<const T*>(role == 0 ? a.k : a.v) + b * a.s0 + h * a.s1;
   for (int i = tid; i < n * kD; i += kAThreads) {
     const int j = i / kD, d = i % kD;
@@ -304,15 +314,26 @@ cudaError_t launch_append(const gtq_plan* p, const void* k, const void* v, const
   a.sm = sm;
   a.cap = p->cfg.t_capacity;
   const dim3 grid((unsigned)p->n_heads, p->cfg.v_bits > 0 ? 2 : 1);  // K-only: keys alone
+  // programmatic dependent launch: the constant prologue overlaps the previous grid
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kAThreads);
+  cfg.dynamicSmemBytes = kRotBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
   if (p->cfg.in_dtype == GTQ_DTYPE_FP16) {
     e = cudaFuncSetAttribute(append_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kRotBytes);
-    if (e == cudaSuccess) append_kernel<__half><<<grid, kAThreads, kRotBytes, s>>>(a);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, append_kernel<__half>, a);
   } else {
     e = cudaFuncSetAttribute(append_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kRotBytes);
-    if (e == cudaSuccess) append_kernel<float><<<grid, kAThreads, kRotBytes, s>>>(a);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, append_kernel<float>, a);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

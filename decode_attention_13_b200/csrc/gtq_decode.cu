@@ -1396,7 +1396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // o_rot^T split into fp16 hi + lo; A_hi B_hi + A_hi B_lo + A_lo B_hi
   for (int mt = warp; mt < 8; mt += blockDim.x >> 5) {
     const int g = lane >> 2, t = lane & 3;
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    // three accumulators (hi.hi, hi.lo, lo.hi), so that the mma chains overlap
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kt = 0; kt < 8; ++kt) {
       const uint4 fh = rvf[((mt * 8 + kt) * 32 + lane) * 2], fl = rvf[((mt * 8 + kt) * 32 + lane) * 2 + 1];
@@ -1412,9 +1413,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t bl1 = pack_half2(__float2half_rn(x1.x - __half2float(h10)),
                                       __float2half_rn(x1.y - __half2float(h11)));
       mma16816(c, ah, bh0, bh1);
-      mma16816(c, ah, bl0, bl1);
-      mma16816(c, al, bh0, bh1);
+      mma16816(c1, ah, bl0, bl1);
+      mma16816(c2, al, bh0, bh1);
     }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) c[r] += c1[r] + c2[r];
     // c[0], c[1]: dim 16 mt + g, heads 2t, 2t + 1; c[2], c[3]: dim + 8
     const int dd = 16 * mt + g;
 #pragma unroll

@@ -200,3 +200,75 @@ def test_argument_checks():
     with pytest.raises(gtq.GtqError):           # coded plans take no fp16 values
         gtq.gtq_decode_attn_full(coded.plan, coded.packed, coded.T, coded.q, out,
                                  kv=gtq.fp16_kv(v=coded.v))
+
+
+def test_key_only_appends_with_window_and_fp32_queries():
+    # K-only plan: widths from a prefix, tokens appended 1, 2 and 4 at a time
+    # (the small-M path), each append followed by a decode on the same stream
+    # with no sync in between; fp32 queries and a window of 24 fp16 rows
+    T_p, W = 600, 24
+    lay = synth.layer((71,), 1, 2, 4, T_p + 7 + W, theta=1e4)
+    k_all, v_all = lay["k"], lay["v"]
+    T = T_p + 7
+    k = torch.from_numpy(np.ascontiguousarray(k_all[:, :, :T])).cuda()
+    v = torch.from_numpy(np.ascontiguousarray(v_all[:, :, :T])).cuda()
+    rk = torch.from_numpy(np.ascontiguousarray(k_all[:, :, T:])).cuda()
+    rv = torch.from_numpy(np.ascontiguousarray(v_all[:, :, T:])).cuda()
+    q32 = torch.from_numpy(lay["q"].astype(np.float32)).cuda()
+    cfg = gtq.make_config(1, 8, 2, 3, 0, T)
+    plan = gtq.gtq_alloc_bits(cfg, k, T_p)
+    packed = torch.zeros(plan.packed_bytes, dtype=torch.uint8, device="cuda")
+    gtq.gtq_quantize_pack(plan, k, None, 0, T_p, packed)
+    kv = gtq.fp16_kv(v=v, recent_k=rk, recent_v=rv)
+    t = T_p
+    for n in (1, 2, 4):
+        gtq.gtq_quantize_pack(plan, k, None, t, n, packed)
+        t += n
+        out = torch.empty((1, 8, 128), dtype=torch.float32, device="cuda")
+        gtq.gtq_decode_attn_full(plan, packed, t, q32, out, kv=kv)
+        torch.cuda.synchronize()
+        ref = np.zeros((1, 8, 128))
+        for h in range(2):
+            bits = allocation.greedy_bits(allocation.block_energy(k_all[0, h, :T_p], 0), 3, 128)
+            kg = quantize.quantize_keys(k_all[0, h, :t], bits, 0)
+            ref[0, 4 * h:4 * h + 4] = attention.decode_general(
+                lay["q"][0, 4 * h:4 * h + 4].astype(np.float32), kg, v_fp16=v_all[0, h, :t],
+                k_recent=k_all[0, h, T:], v_recent=v_all[0, h, T:])
+        assert rel_l2(out.cpu().numpy(), ref) <= DECODE_REL_L2, t
+    assert gtq.gtq_status(plan) == gtq.GTQ_OK
+
+
+def test_key_only_paged_pool_with_mixed_lengths():
+    # K-only keys in a paged pool (pages in reversed order), fp16 values read
+    # by token from the caller's tensor, sequences of their own lengths
+    B, hkv, gq, T = 3, 2, 4, 450
+    lens = [450, 130, 1]
+    lay = synth.layer((72,), B, hkv, gq, T, theta=1e4)
+    k = torch.from_numpy(lay["k"]).cuda()
+    v = torch.from_numpy(lay["v"]).cuda()
+    q = torch.from_numpy(lay["q"]).cuda()
+    n_tiles = (T + 63) // 64
+    pages = B * n_tiles
+    table = torch.arange(pages - 1, -1, -1, dtype=torch.int32, device="cuda").view(B, n_tiles)
+    seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    lay_ = gtq.seq_layout(seq, table)
+    cfg = gtq.make_config(B, hkv * gq, hkv, 3, 0, T)
+    plan = gtq.gtq_alloc_bits_ex(cfg, k, T, layout=gtq.seq_layout(seq))
+    tb = gtq.gtq_layout_tile_bytes(3, 0)
+    pool = torch.zeros(pages * hkv * tb, dtype=torch.uint8, device="cuda")
+    gtq.gtq_quantize_pack_ex(plan, k, None, 0, T, pool, layout=lay_)
+    out = torch.empty((B, hkv * gq, 128), dtype=torch.float32, device="cuda")
+    gtq.gtq_decode_attn_full(plan, pool, T, q, out, layout=lay_, kv=gtq.fp16_kv(v=v))
+    torch.cuda.synchronize()
+    bits_gpu = gtq.gtq_get_bits(plan)
+    ref = np.zeros((B, hkv * gq, 128))
+    for b in range(B):
+        for h in range(hkv):
+            kk = lay["k"][b, h, :lens[b]]
+            bits = allocation.greedy_bits(allocation.block_energy(kk, 0), 3, 128)
+            assert np.array_equal(bits_gpu[b, h].astype(np.int64), bits), (b, h)
+            kg = quantize.quantize_keys(kk, bits, 0)
+            ref[b, h * gq:(h + 1) * gq] = attention.decode_general(
+                lay["q"][b, h * gq:(h + 1) * gq], kg, v_fp16=lay["v"][b, h, :lens[b]])
+    assert rel_l2(out.cpu().numpy(), ref) <= DECODE_REL_L2
+    assert gtq.gtq_status(plan) == gtq.GTQ_OK
