@@ -66,7 +66,7 @@ constexpr uint32_t kOffFlags = kOffLut + (uint32_t)kCodeLutBytes;  // uint8 [2][
 constexpr uint32_t kOffMeta = kOffFlags + 16;
 constexpr uint32_t kOffInfo = kOffMeta + ((sizeof(HeadMeta) + 15) & ~15);
 constexpr uint32_t kOffBar = kOffInfo + 512;
-constexpr int kNumBars = 17;
+constexpr int kNumBars = 18;
 constexpr uint32_t kTcSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slack for 1024-byte alignment
 static_assert(kOffP % 1024 == 0 && kOffA % 1024 == 0, "swizzled operands need 1024-byte alignment");
 static_assert(kTcSmem <= 232448, "shared memory budget");
@@ -81,6 +81,7 @@ constexpr int kCEmpty = 10;  // [2] code accumulator read by the 8 code warps
 constexpr int kSFull = 12;   // [2] scales of a tile written by the 4 norm warps
 constexpr int kSEmpty = 14;  // [2] scales read by the 8 code warps
 constexpr int kRBar = 16;    // R image loaded
+constexpr int kDrain = 17;   // after a failed wait: the MMAs issued so far are done
 
 // per-CTA gather layout (built once)
 struct GatherInfo {
@@ -353,6 +354,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     }
     mbar_init(bar(kPFull), 1);
     mbar_init(bar(kPEmpty), 4);
+    mbar_init(bar(kDrain), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kCFull + i), 1);
       mbar_init(bar(kCEmpty + i), 8);
@@ -425,7 +427,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
   const uint32_t tmem = *tmem_slot;
 
   const int64_t n_mt = a.mt1 - a.mt0;
-  int failed = 0;
+  int failed = 0, issued = 0;  // issued: tile copies the producer started
   if (warp == 0) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
@@ -436,6 +438,7 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
       for (int64_t t = cta; t < n_mt; t += n_cta, ++it) {
         const int st = it % kStages;
         if (!mbar_wait(bar(kEmpty + st), ((it / kStages) & 1) ^ 1)) { failed = 1; break; }
+        issued = it + 1;
         const uint32_t dst = sb + kOffA + st * kStageBytes;
         const int row = (int)((a.mt0 + t) * kMTile);
         mbar_expect_tx(bar(kFull + st), kStageBytes);
@@ -718,6 +721,20 @@ __device__ __forceinline__ void tc_role(const CUtensorMap* tmap, const TcArgs& a
     }
   }
   if (failed) atomicOr(a.status, kStatusTimeout);
+  // After a failed wait, nothing in flight may outlive the CTA: the MMA issuer
+  // waits (bounded) until its issued MMAs are done, the producer until every
+  // tile copy it issued has landed.  Otherwise every copy and MMA was consumed.
+  if (__syncthreads_or(failed)) {
+    if (warp == 1 && lane == 0) {
+      tc_commit(bar(kDrain));
+      mbar_wait(bar(kDrain), 0);
+    }
+    if (warp == 0 && lane == 0)
+      for (int st = 0; st < kStages && st < issued; ++st) {
+        const int last = st + ((issued - 1 - st) / kStages) * kStages;  // last fill of the stage
+        mbar_wait(bar(kFull + st), (last / kStages) & 1);
+      }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
