@@ -166,6 +166,9 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr)
                : "memory");
 }
+__device__ __forceinline__ void prefetch_l2(const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // the packed cache is streamed once per call: evicted first, so that it does
 // not push the tables and metadata out of L2
 __device__ __forceinline__ uint64_t evict_first_policy() {
@@ -465,13 +468,15 @@ __device__ bool arrive_last(unsigned* ticket, unsigned count, int* flag) {
 // Merge partials [first, first + count) (count <= kMergeGroup) of the 8 query
 // heads: M = max m_j, L = sum 2^(m_j - M) l_j, o = sum 2^(m_j - M) o_j.  Written
 // as a partial to dst (global) or, normalised (o / L), to o_rot (shared) with
-// (M, L) to hm / hl.  Warp hh (< 8) takes query head hh, lane = 4 dims: whole
+// (M, L) to hm / hl.  Warp w0 + i takes query head i (and i + warps), lane = 4 dims: whole
 // partial rows (coalesced), every load in flight at once, one pass.  Partials
 // come from other CTAs: loads bypass L1.  The caller synchronises afterwards.
 __device__ __noinline__ void merge_partials(const float* head_parts, int first, int count,
-                                            float* dst, float (*o_rot)[kD], float* hm, float* hl) {
+                                            float* dst, float (*o_rot)[kD], float* hm, float* hl,
+                                            int w0 = 0) {
   const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int hh = threadIdx.x >> 5; hh < 8; hh += nwarps) {
+  // warp w0 takes head 0: two merges with different w0 run side by side
+  for (int hh = ((threadIdx.x >> 5) - w0 % nwarps + nwarps) % nwarps; hh < 8; hh += nwarps) {
     float2 ml[kMergeGroup];
     float4 oj[kMergeGroup];
 #pragma unroll
@@ -816,6 +821,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
 
+  // the window rows this split will attend after its tiles: into L2 now
+  const int64_t wl = window_len(a.rlens, a.rlen, b);
+  const int n_w = (int)min((int64_t)min(nsplit, kWindowPartials), (wl + 31) / 32);
+  if (producer && lane == 0 && split < n_w && a.rs2 == kD)
+    for (int64_t r0 = 32 * (int64_t)split; r0 < wl; r0 += 32 * (int64_t)n_w) {
+      const unsigned bytes = (unsigned)(min((int64_t)32, wl - r0) * kD * 2);
+      prefetch_l2(a.rk + b * a.rs0 + h * a.rs1 + r0 * kD, bytes);
+      prefetch_l2(a.rv + b * a.rs0 + h * a.rs1 + r0 * kD, bytes);
+    }
   if (producer) {
     // ------------------------------------------------------------ producer
     // The whole warp runs the schedule (lane 0's counter grabs are broadcast);
@@ -1308,8 +1322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // the first n_w splits also attend the fp16 window's 32-row blocks, each
   // into a window partial of its own, before their arrival publishes it
-  const int64_t wl = window_len(a.rlens, a.rlen, b);
-  const int n_w = (int)min((int64_t)min(nsplit, kWindowPartials), (wl + 31) / 32);
   if (split < n_w) {
     const WindowArgs wa = {a.q, a.rk, a.rv, a.rs0, a.rs1, a.rs2, a.q_fp32, a.hkv, a.gq};
     window_pass(wa, s, b, h, split, n_w, wl, ncw, stages, stage_sa,
@@ -1328,10 +1340,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return true;
   };
+  // the window's partials merged into qb (normalised) with (M_w, L_w) in wsc[0],
+  // [1], by other warps than the cache's merge (no barrier between the two)
+  auto merge_window = [&]() {
+    if (n_w > 0) merge_partials(head_parts, a.slot_window, n_w, nullptr, s.qb, s.wsc[0], s.wsc[1], 8);
+  };
   bool finish = nsplit == 1, rv_issued = false;
   if (finish) {
     __syncthreads();
     rv_issued = fetch_rv();
+    merge_window();
   } else {
     const int n_grp = (nsplit + kMergeGroup - 1) / kMergeGroup;
     const int grp = split / kMergeGroup;
@@ -1340,6 +1358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       rv_issued = fetch_rv();
       if (n_grp == 1) {
         merge_partials(head_parts, grp * kMergeGroup, n1, nullptr, s.qa, s.hm, s.hl);
+        merge_window();
         finish = true;
       } else {
         merge_partials(head_parts, grp * kMergeGroup, n1,
@@ -1347,6 +1366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        s.hm, s.hl);
         if (arrive_last(&head_tickets[0], (unsigned)n_grp, &s.flag)) {
           merge_partials(head_parts, a.slot_groups, n_grp, nullptr, s.qa, s.hm, s.hl);
+          merge_window();
           finish = true;
         }
       }
@@ -1361,11 +1381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!rv_ok) {
     if (tid == 0) atomicOr(a.status, kStatusTimeout);
     return;
-  }
-  // the window's partials merged into qb (normalised) with (M_w, L_w) in wsc[0], [1]
-  if (n_w > 0) {
-    merge_partials(head_parts, a.slot_window, n_w, nullptr, s.qb, s.wsc[0], s.wsc[1]);
-    __syncthreads();
   }
   // out = cr o_cache + cw o_window (both normalised): the two softmax parts
   // weighted by their sums at their common maximum
@@ -1518,7 +1533,11 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   if (area < kTailBytes || area < kPackArea + a.stride) return cudaErrorInvalidValue;
   const int ring = std::min(kMaxRing, area / a.stride);
   if (ring < 2) return cudaErrorInvalidValue;
-  const int np = std::max(1, std::min(kPairs, ring * kTPS / 2));
+  // pairs: half the tile slots (each pair has its next tile in flight); K-only
+  // stages are large (fp16 value rows), so there one pair per slot (measured
+  // 22% faster at 128K; pairs take slots in order, so the producer always
+  // advances)
+  const int np = std::max(1, std::min(kPairs, konly ? ring * kTPS : ring * kTPS / 2));
   a.ring = ring;
   a.np = np;
   const int64_t tiles_T = (T + kTile - 1) / kTile;
