@@ -241,6 +241,7 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
 struct DecodeSmem {
   alignas(16) HeadMeta meta;
   uint4 qf[kMaxKt][32];        // per k-tile & lane: hi(slot A), hi(slot B), lo(A), lo(B)
+  uint4 wqf[8][32];            // the window's q fragments (original basis): hi, hi, lo, lo
   alignas(16) float qa[8][kD];  // gathered queries [coordinate][head], then the merged o_rot
   alignas(16) float qb[8][kD];  // the raw queries (bulk copy), then q_rot (scaled)
   uint4 gdesc[kMaxGroups];      // W | split << 4 | k16 tiles << 8 | half k-tile << 16; key
@@ -541,17 +542,15 @@ struct HeadView {
 // basis.
 constexpr int kWinRowBytes = 2 * kD + 16;
 constexpr int kWinBufBytes = 2 * 32 * kWinRowBytes;  // K and V rows of one block
-constexpr int kWinWarps = 4;
+constexpr int kWinWarps = 3;
 constexpr int kWinBytes = kWinWarps * kWinBufBytes + kWinWarps * 8 * kWoStride * 4;
-static_assert(kWinBytes <= kTailBytes, "window staging fits in the merge area");
+static_assert(kWinBytes <= kPackArea, "window staging fits in the rotation pack's area");
 static_assert(kWindowPartials <= kMergeGroup, "window partials merge in one pass");
 
 struct WindowArgs {
-  const void* q;
   const __half* rk;
   const __half* rv;
   int64_t rs0, rs1, rs2;
-  int q_fp32, hkv, gq;
 };
 
 // Window rows of sequence b (clamped to [0, rlen]).
@@ -560,33 +559,24 @@ __device__ __forceinline__ int64_t window_len(const int32_t* rlens, int rlen, in
   return rlens ? min(max((int64_t)rlens[b], (int64_t)0), (int64_t)rlen) : (int64_t)rlen;
 }
 
-// This split's window blocks j = split + k n_w (32 rows each) -> partial
-// (m, l, o) of the 8 query heads at dst, in the layout of a split's partial.
-// Every thread of the CTA calls it; it uses the stage area, qf and the warp
-// tables, and leaves qa, hm and hl alone.
-__device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int b, int h,
-                                         int split, int n_w, int64_t wl, int ncw, uint8_t* area,
-                                         uint32_t area_sa, float* dst) {
-  __syncthreads();  // the stage area and the warp tables are free
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int nww = min(ncw, kWinWarps);
-  // B fragments of q in the original basis, times log2(e) / sqrt(d): fp16 hi, lo
-  const float qs = 1.4426950408889634f * 0.08838834764831845f;
-  for (int idx = tid; idx < 8 * 32; idx += blockDim.x) {
+// The window's B fragments of q in the original basis, times log2(e) / sqrt(d),
+// as fp16 hi and lo, from the raw queries in qb (consumer threads).
+__device__ __noinline__ void window_fragments(DecodeSmem& s, int q_fp32, int gq, int nct) {
+  const float qs = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+  for (int idx = threadIdx.x; idx < 8 * 32; idx += nct) {
     const int kt = idx >> 5, ln = idx & 31, gg = ln >> 2, tt = ln & 3;
     uint32_t o4[4];
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int d = 16 * kt + 2 * tt + 8 * hf;
+      const int d = (gg << 7) | (16 * kt + 2 * tt + 8 * hf);
       float v0 = 0.f, v1 = 0.f;
-      if (gg < a.gq) {
-        const size_t qi = (((size_t)b * a.hkv + h) * a.gq + gg) * kD + d;
-        if (a.q_fp32) {
-          v0 = reinterpret_cast<const float*>(a.q)[qi];
-          v1 = reinterpret_cast<const float*>(a.q)[qi + 1];
+      if (gg < gq) {
+        if (q_fp32) {
+          v0 = (&s.qb[0][0])[d];
+          v1 = (&s.qb[0][0])[d + 1];
         } else {
-          v0 = __half2float(reinterpret_cast<const __half*>(a.q)[qi]);
-          v1 = __half2float(reinterpret_cast<const __half*>(a.q)[qi + 1]);
+          v0 = __half2float(reinterpret_cast<const __half*>(&s.qb[0][0])[d]);
+          v1 = __half2float(reinterpret_cast<const __half*>(&s.qb[0][0])[d + 1]);
         }
       }
       v0 *= qs;
@@ -595,9 +585,21 @@ __device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int 
       o4[hf] = pack_half2(h0, h1);
       o4[2 + hf] = pack_half2(__float2half_rn(v0 - __half2float(h0)), __float2half_rn(v1 - __half2float(h1)));
     }
-    s.qf[kt][ln] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    s.wqf[kt][ln] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
   }
-  __syncthreads();
+}
+
+// This split's window blocks j = split + k n_w (32 rows each) -> partial
+// (m, l, o) of the 8 query heads at dst, in the layout of a split's partial.
+// Every consumer thread calls it during setup, after the query rotation: it
+// stages rows in `area` (the rotation pack's area, free by then and not yet
+// handed to the producer), reads the window's q fragments (wqf) and uses the
+// warp tables.
+__device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int b, int h,
+                                         int split, int n_w, int64_t wl, int ncw, uint8_t* area,
+                                         uint32_t area_sa, float* dst) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int nct = ncw * 32, nww = min(ncw, kWinWarps);
   float* wo2 = reinterpret_cast<float*>(area + kWinWarps * kWinBufBytes);  // [warp][head][kWoStride]
   if (warp < nww) {
     uint8_t* kbuf = area + warp * kWinBufBytes;
@@ -638,7 +640,7 @@ __device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int 
                        : "=r"(av[0]), "=r"(av[1]), "=r"(av[2]), "=r"(av[3])
                        : "r"(arow + (uint32_t)((2 * kt + (lane >> 4)) * 16))
                        : "memory");
-          const uint4 qv = s.qf[kt][lane];
+          const uint4 qv = s.wqf[kt][lane];
           mma16816(S_[mt], av, qv.x, qv.y);
           mma16816(S_[mt], av, qv.z, qv.w);
         }
@@ -718,7 +720,7 @@ __device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int 
       o0[kWoStride + 16 * i + g + 8] = O[i][3];
     }
   }
-  __syncthreads();
+  consumers_sync(nct);
   if (tid < 8) {
     const int hh = tid;
     float M = -1e30f;
@@ -731,8 +733,8 @@ __device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int 
     }
     *reinterpret_cast<float2*>(dst + hh * kPartialStride) = make_float2(M, L);
   }
-  __syncthreads();
-  for (int idx = tid; idx < 8 * kD / 4; idx += blockDim.x) {
+  consumers_sync(nct);
+  for (int idx = tid; idx < 8 * kD / 4; idx += nct) {
     const int hh = idx >> 5, d4 = idx & 31;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int w = 0; w < nww; ++w) {
@@ -745,6 +747,7 @@ __device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int 
     }
     *reinterpret_cast<float4*>(dst + hh * kPartialStride + 4 + 4 * d4) = v;
   }
+  consumers_sync(nct);  // the staging area is free again
 }
 
 template <int VB>
@@ -815,11 +818,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned* head_tickets = a.tickets + (size_t)head * kTicketStride;
   bool failed = false;
 
-  // per-warp running state (consumers)
+  // per-warp running state (consumers; set just before the tile loop)
   float mrun[2] = {-1e30f, -1e30f}, lrun[2] = {0.f, 0.f};
   float O[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
 
   // the window rows this split will attend after its tiles: into L2 now
   const int64_t wl = window_len(a.rlens, a.rlen, b);
@@ -991,6 +992,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       qT[p][hh] = v;
     }
+    if (split < n_w) window_fragments(s, a.q_fp32, a.gq, nct);  // before the rotation overwrites qb
     consumers_sync(nct);
     // q_rot[hh][pos] = sum_c R_g[r][c] qT[first + c][hh] * log2(e) / (sqrt(d) sqrt(m_g)),
     // into qb: a task is one position and four heads
@@ -1022,6 +1024,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       s.qb[h4 + 3][pos] = acc.w * sc;
     }
     consumers_sync(nct);
+    // the first n_w splits attend the fp16 window's 32-row blocks now, staged in
+    // the pack's area, each into a window partial of its own
+    if (split < n_w) {
+      const WindowArgs wa = {a.rk, a.rv, a.rs0, a.rs1, a.rs2};
+      window_pass(wa, s, b, h, split, n_w, wl, ncw, reinterpret_cast<uint8_t*>(pack), smem_u32(pack),
+                  a.partials + ((size_t)head * a.slot_total + a.slot_window + split) * 8 * kPartialStride);
+    }
     if (tid == 0) mbar_arrive(&s.done_bar);  // the pack's stages may be filled now
     // group descriptors: W | split << 4 | k16 tiles << 8 | half k-tile << 16
     if (tid < m.n_groups) {
@@ -1062,6 +1071,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // lane portion of slot t: 16W bits at byte 16W t + 2W g; this warp's half: + W wh
     const int lane_kunit = 16 * t + 2 * g + wh;  // times W
 
+#pragma unroll
+    for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
     // tile slot j = pair + k np of the stage sequence: stage j / kTPS, slot j % kTPS
     int j = pair, fi = pair / kTPS, slot = fi % S, round = fi / S;
     // a timeout seen by any lane stops the whole warp (the loop body is warp-wide)
@@ -1319,13 +1330,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<float4*>(part + hh * kPartialStride + 4 + 4 * d4) = v;
       if (d4 == 0) *reinterpret_cast<float2*>(part + hh * kPartialStride) = make_float2(s.hm[hh], s.hl[hh]);
     }
-  }
-  // the first n_w splits also attend the fp16 window's 32-row blocks, each
-  // into a window partial of its own, before their arrival publishes it
-  if (split < n_w) {
-    const WindowArgs wa = {a.q, a.rk, a.rv, a.rs0, a.rs1, a.rs2, a.q_fp32, a.hkv, a.gq};
-    window_pass(wa, s, b, h, split, n_w, wl, ncw, stages, stage_sa,
-                head_parts + (size_t)(a.slot_window + split) * 8 * kPartialStride);
   }
   // ---------------- merge of the splits, without waiting: the last CTA to
   // arrive in a group of kMergeGroup splits merges the group into a
