@@ -750,7 +750,9 @@ __device__ __noinline__ void window_pass(const WindowArgs a, DecodeSmem& s, int 
   consumers_sync(nct);  // the staging area is free again
 }
 
-template <int VB>
+// WIN: a window of fp16 rows may be attended (a separate instantiation, so that
+// decodes without one carry none of its code)
+template <int VB, bool WIN>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap vmap, DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -822,9 +824,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   float mrun[2] = {-1e30f, -1e30f}, lrun[2] = {0.f, 0.f};
   float O[8][4];
 
-  // the window rows this split will attend after its tiles: into L2 now
-  const int64_t wl = window_len(a.rlens, a.rlen, b);
-  const int n_w = (int)min((int64_t)min(nsplit, kWindowPartials), (wl + 31) / 32);
+  // the window rows this split will attend: into L2 now
+  const int64_t wl = WIN ? window_len(a.rlens, a.rlen, b) : 0;
+  const int n_w = WIN ? (int)min((int64_t)min(nsplit, kWindowPartials), (wl + 31) / 32) : 0;
   if (producer && lane == 0 && split < n_w && a.rs2 == kD)
     for (int64_t r0 = 32 * (int64_t)split; r0 < wl; r0 += 32 * (int64_t)n_w) {
       const unsigned bytes = (unsigned)(min((int64_t)32, wl - r0) * kD * 2);
@@ -1554,10 +1556,17 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   switch (p->cfg.v_bits) {
 #define GTQ_LAUNCH_VB(VB)                                                                     \
   case VB:                                                                                   \
-    e = cudaFuncSetAttribute(decode_kernel<VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             kSmemBytes);                                                     \
-    if (e == cudaSuccess)                                                                    \
-      e = launch_pdl(decode_kernel<VB>, grid, block, kSmemBytes, s, vmap, a);                 \
+    if (a.rlen > 0) {                                                                        \
+      e = cudaFuncSetAttribute(decode_kernel<VB, true>,                                      \
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);     \
+      if (e == cudaSuccess)                                                                  \
+        e = launch_pdl(decode_kernel<VB, true>, grid, block, kSmemBytes, s, vmap, a);        \
+    } else {                                                                                 \
+      e = cudaFuncSetAttribute(decode_kernel<VB, false>,                                     \
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);     \
+      if (e == cudaSuccess)                                                                  \
+        e = launch_pdl(decode_kernel<VB, false>, grid, block, kSmemBytes, s, vmap, a);       \
+    }                                                                                        \
     break;
     GTQ_LAUNCH_VB(0)
     GTQ_LAUNCH_VB(1) GTQ_LAUNCH_VB(2) GTQ_LAUNCH_VB(3) GTQ_LAUNCH_VB(4)
