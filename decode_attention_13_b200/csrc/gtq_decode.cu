@@ -4,16 +4,17 @@
 // tensor-core operands in registers.  One launch per call (decode_kernel),
 // grid = (heads, splits), one CTA per SM, 2 * np consumer warps (np pairs) and
 // one producer warp:
-//   setup    before the grid-dependency wait: the constant lookup tables
-//            (bulk copy; an L2 prefetch of the CTA's tiles there measured 8%
-//            slower over a 36-layer step); after it: the head metadata, the key
-//            rotation blocks and the queries, then q_rot = M_h q for the 8 query heads of the KV head,
-//            from each group's m x m block only, times log2(e) / (sqrt(d)
-//            sqrt(m_g)), and its fp16 hi / lo MMA fragments.
-//   loop     the producer takes tiles from a per-head counter (two at a time,
-//            the next grab in flight while the current one is used) and
-//            bulk-copies each 64-token tile into a ring of stages; the pair
-//            that owns a stage splits it, 32 tokens per warp.  Scores:
+//   setup    before the grid-dependency wait: the constant lookup tables (bulk
+//            copy; an L2 prefetch of the CTA's tiles there measured 8% slower
+//            over a 36-layer step).  After it: the head metadata, the key
+//            rotation blocks and the queries by bulk copy; q_rot = M_h q for
+//            the 8 query heads of the KV head, from each group's m x m block
+//            only, times log2(e) / (sqrt(d) sqrt(m_g)); its fp16 hi / lo MMA
+//            fragments.
+//   loop     the producer deals 7/8 of a head's tiles statically and the rest
+//            from a per-head counter (two at a time, the next grab in flight),
+//            and bulk-copies two adjacent 64-token tiles per stage into a ring;
+//            the pair that owns a tile splits it, 32 tokens per warp.  Scores:
 //            mma.m16n8k16 (m16n8k8 for a group's last half k-tile) with
 //            A = codebook values of 16 tokens x 16 rotated coords (pair tables)
 //            and B = q_rot, per key group, scaled by the group's fp16 norms;
@@ -23,17 +24,19 @@
 //            B = P^T (movmatrix transpose of the score fragment), in V's
 //            rotated basis.
 //   merge    the CTA's warps, then the splits: the last CTA of each group of
-//            16 splits merges the group (and fetches R_V), the last group
-//            merges the rest and writes o = R_V^T o_rot / l.  Tickets and the
-//            tile counter return to 0 for the next call.
+//            16 splits merges the group (and fetches R_V^T's fragments), the
+//            last group merges the rest and writes o = R_V^T o_rot / l with
+//            mma (fp16 hi / lo parts).  Tickets and the tile counter return to
+//            0 for the next call.
 // K-only plans (values kept in fp16, the page's K-only quantization, Abstract)
-// take decode_kernel<0>: each stage also receives the tiles' fp16 value rows
+// take decode_kernel<0, *>: each stage also receives the tiles' fp16 value rows
 // by a tensor copy (128-byte swizzle, so that the transposing ldmatrix that
 // forms A = V^T is free of bank conflicts), P.V runs in the original basis and
 // no R_V^T product follows.  An fp16 window of recent tokens (the recent-key
-// buffer the page's method does without, Abstract) is attended by split 0 on
-// the CUDA cores into a partial of its own, combined with the cache's (m, l)
-// by the CTA that finishes the head.
+// buffer the page's method does without, Abstract) is attended, in the
+// decode_kernel<*, true> instantiations, by the first splits during setup on
+// the tensor cores, each into a partial of its own; the finishing CTA merges
+// those and combines them with the cache's part by their softmax sums.
 #include <algorithm>
 #include <climits>
 #include <cmath>

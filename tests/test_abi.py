@@ -132,3 +132,62 @@ def test_status_helpers_reject_null_plan():
     lib = gtq.binding._lib
     assert lib.gtq_raise_status(None, gtq.GTQ_ERR_TIMEOUT) == gtq.GTQ_ERR_INVALID
     assert lib.gtq_plan_device_bytes(None) == 0
+
+
+def test_key_only_tile_bytes_and_reader_agree():
+    from tests import layout
+
+    for kb in range(1, 9):
+        assert gtq.gtq_layout_tile_bytes(kb, 0) == 1024 * kb + 1024 == layout.tile_bytes(kb, 0)
+        for vb in range(1, 9):
+            assert gtq.gtq_layout_tile_bytes(kb, vb) == layout.tile_bytes(kb, vb)
+    assert gtq.gtq_layout_tile_bytes(3, 9) == 0 and gtq.gtq_layout_tile_bytes(3, -1) == 0
+
+
+def test_null_plan_calls_of_the_layout_entry_points():
+    lib = gtq.binding._lib
+    st = (ctypes.c_int64 * 4)(0, 0, 128, 1)
+    lay = gtq.binding.gtq_seq_layout(None, None, 0)
+    kv = gtq.binding.gtq_fp16_kv()
+    out = ctypes.c_void_p()
+    assert lib.gtq_alloc_bits_ex(None, 0x1000, 1, st, ctypes.byref(lay), None,
+                                 ctypes.byref(out)) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_quantize_pack_ex(None, 0x1000, 0x1000, st, 0, 1, 0x1000, 1 << 20,
+                                    ctypes.byref(lay), None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_decode_attn_ex(None, 0x1000, 1, ctypes.byref(lay), 0x1000, 0, 0x1000,
+                                  None) == gtq.GTQ_ERR_INVALID
+    assert lib.gtq_decode_attn_full(None, 0x1000, 1, None, ctypes.byref(kv), 0x1000, 0, 0x1000,
+                                    None) == gtq.GTQ_ERR_INVALID
+
+
+def test_struct_layouts_match_the_header():
+    # the binding's ctypes structs against the C compiler's view of include/gtq.h
+    import shutil
+    import subprocess
+    import tempfile
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = {
+        "gtq_config": [f for f, _ in gtq.binding.gtq_config._fields_],
+        "gtq_seq_layout": [f for f, _ in gtq.binding.gtq_seq_layout._fields_],
+        "gtq_fp16_kv": [f for f, _ in gtq.binding.gtq_fp16_kv._fields_],
+    }
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "gtq.h"', 'int main(void) {']
+    for st, fs in fields.items():
+        lines.append('printf("%s %%zu\\n", sizeof(%s));' % (st, st))
+        for f in fs:
+            lines.append('printf("%s.%s %%zu\\n", offsetof(%s, %s));' % (st, f, st, f))
+    lines += ['return 0;', '}']
+    with tempfile.TemporaryDirectory() as d:
+        src, exe = os.path.join(d, "t.c"), os.path.join(d, "t")
+        open(src, "w").write("\n".join(lines))
+        subprocess.run([cc, "-I", os.path.join(ROOT, "include"), src, "-o", exe], check=True)
+        got = dict(l.split() for l in subprocess.run([exe], capture_output=True, text=True,
+                                                    check=True).stdout.split("\n") if l)
+    for st, fs in fields.items():
+        cls = getattr(gtq.binding, st)
+        assert int(got[st]) == ctypes.sizeof(cls), st
+        for f in fs:
+            assert int(got["%s.%s" % (st, f)]) == getattr(cls, f).offset, (st, f)
