@@ -139,3 +139,63 @@ def test_full_size_layer(config):
         ok, ov = _check_head_codes(head, bits, kb, vb, T, k_np, v_np, config * 1000 + b * 10 + h)
         ref = attention.decode_rotated(q_np, ok, ov)
         assert _rel_l2(out_np[b, h * gq:(h + 1) * gq], ref) <= DECODE_REL_L2, (b, h)
+
+
+def test_full_size_key_only_with_window():
+    # the headline layer's shape (T = 131072, 16q/2kv) as a K-only plan (keys
+    # coded at 3 bits, values read in fp16) with a 128-row fp16 window, decoded
+    # in one gtq_decode_attn_full call as the bench's variants do; every head
+    # checked: widths, sampled key codes and norms, and the output against the
+    # oracle's decode of the library's own key codes, the fp16 values and the
+    # window rows
+    c = synth.CONFIGS[2]
+    B, hq, hkv, T, kb, W = c["B"], c["h_q"], c["h_kv"], c["T"], c["k_bits"], 128
+    gq = hq // hkv
+    k, v, q = synth.layer_torch((2, 0, 0), B, hkv, gq, T, theta=c["theta"], decay=c["decay"],
+                                device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    rk = torch.randn((B, hkv, W, 128), generator=gen, device="cuda", dtype=torch.float16)
+    rv = torch.randn((B, hkv, W, 128), generator=gen, device="cuda", dtype=torch.float16)
+    torch.cuda.synchronize()
+    plan = gtq.gtq_alloc_bits(gtq.make_config(B, hq, hkv, kb, 0, T), k, T)
+    packed = torch.empty(plan.packed_bytes, dtype=torch.uint8, device="cuda")
+    gtq.gtq_quantize_pack(plan, k, None, 0, T, packed)
+    out = torch.empty((B, hq, 128), dtype=torch.float32, device="cuda")
+    gtq.gtq_decode_attn_full(plan, packed, T, q, out,
+                             kv=gtq.fp16_kv(v=v, recent_k=rk, recent_v=rv))
+    torch.cuda.synchronize()
+    assert gtq.gtq_status(plan) == gtq.GTQ_OK
+    bits_gpu = gtq.gtq_get_bits(plan)
+    per = plan.packed_bytes // (B * hkv)
+    out_np = out.cpu().numpy()
+    for h in range(hkv):
+        k_np = k[0, h].cpu().numpy()
+        _, bits = _oracle_bits(k_np, kb)
+        assert np.array_equal(bits_gpu[0, h].astype(np.int64), bits), h
+        keys, vcodes, vnorm = layout.read_head(packed[h * per:(h + 1) * per].cpu().numpy(), bits,
+                                               kb, 0, T)
+        assert vcodes is None and vnorm is None
+        rng = np.random.default_rng(77 + h)
+        idx = np.unique(np.concatenate([np.arange(64), np.arange(T - 64, T),
+                                        rng.choice(T, SAMPLE_TOKENS, replace=False)]))
+        kg = quantize.quantize_keys(k_np[idx], bits, 0)
+        by_w = {g.width: g for g in kg}
+        flips = total = 0
+        for (w, codes, n16) in keys:
+            og = by_w[w]
+            d = codes[idx] - og.codes
+            assert np.all(np.abs(d) <= 1)
+            flips += int(np.count_nonzero(d))
+            total += d.size
+            nd = (n16[idx].view(np.uint16).astype(np.int64)
+                  - og.norm16.view(np.uint16).astype(np.int64))
+            assert np.all(np.abs(nd) <= 1)
+        assert flips <= CODE_FLIP_MAX * total, (flips, total)
+        coords = {g.width: g.coords for g in kg}
+        ok = [quantize.CodedGroup(w, coords[w], cc, n, n.astype(np.float64), False)
+              for (w, cc, n) in keys]
+        ref = attention.decode_general(q[0, h * gq:(h + 1) * gq].float().cpu().numpy(), ok,
+                                       v_fp16=v[0, h].cpu().numpy(),
+                                       k_recent=rk[0, h].cpu().numpy(),
+                                       v_recent=rv[0, h].cpu().numpy())
+        assert _rel_l2(out_np[0, h * gq:(h + 1) * gq], ref) <= DECODE_REL_L2, h
