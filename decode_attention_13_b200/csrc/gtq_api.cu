@@ -72,6 +72,8 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   p->n_heads = cfg->batch * cfg->n_kv_heads;
   p->n_blocks = cfg->head_dim / 2;
   p->g_q = cfg->n_q_heads / cfg->n_kv_heads;
+  p->n_qs = (p->g_q + kQSlice - 1) / kQSlice;
+  p->n_units = p->n_heads * p->n_qs;
   p->n_tiles = (cfg->t_capacity + kTile - 1) / kTile;
   p->tile_bytes = gtq_layout_tile_bytes(cfg->k_bits, cfg->v_bits);
   p->packed_bytes = (size_t)p->n_heads * p->n_tiles * p->tile_bytes;
@@ -91,11 +93,12 @@ int make_plan(const gtq_config* cfg, gtq_plan** out) {
   alloc((void**)&p->d_mrow, H * kD * kD * sizeof(float));
   alloc((void**)&p->d_rotpack, H * kRotPackBytes);
   if (cfg->head_dim == kD) alloc((void**)&p->d_bimg, H * b_image_bytes());
-  alloc((void**)&p->d_partials, H * (size_t)PartialSlots(decode_split_cap(p->n_sms, p->n_heads)).total *
+  const size_t U = p->n_units;
+  alloc((void**)&p->d_partials, U * (size_t)PartialSlots(decode_split_cap(p->n_sms, p->n_units)).total *
                                     8 * kPartialStride * sizeof(float));
-  alloc((void**)&p->d_tickets, H * kTicketStride * sizeof(unsigned));
+  alloc((void**)&p->d_tickets, U * kTicketStride * sizeof(unsigned));
   alloc((void**)&p->d_status, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, H * kTicketStride * sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemset(p->d_tickets, 0, U * kTicketStride * sizeof(unsigned));
   if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(p->d_meta, 0, H * sizeof(HeadMeta));
   if (e != cudaSuccess) {
@@ -313,12 +316,12 @@ int gtq_get_energy(gtq_plan* plan, double* host_energy, void* stream) {
 
 size_t gtq_plan_device_bytes(const gtq_plan* plan) {
   if (!plan) return 0;
-  const size_t H = plan->n_heads;
+  const size_t H = plan->n_heads, U = plan->n_units;
   size_t b = H * plan->n_blocks * sizeof(double) + H * plan->n_blocks + H * sizeof(HeadMeta) +
              H * kD * kD * sizeof(float) + H * kRotPackBytes +
-             H * (size_t)PartialSlots(decode_split_cap(plan->n_sms, plan->n_heads)).total * 8 *
+             U * (size_t)PartialSlots(decode_split_cap(plan->n_sms, plan->n_units)).total * 8 *
                  kPartialStride * sizeof(float) +
-             H * kTicketStride * sizeof(unsigned) + sizeof(int);
+             U * kTicketStride * sizeof(unsigned) + sizeof(int);
   if (plan->cfg.head_dim == kD) b += H * b_image_bytes();
   return b;
 }

@@ -2,13 +2,15 @@
 // Allocation for KV-Cache Quantization", Abstract: decoding is served straight
 // from the packed cache).  No fp16 K or V is materialised: codes become
 // tensor-core operands in registers.  One launch per call (decode_kernel),
-// grid = (heads, splits), one CTA per SM, 2 * np consumer warps (np pairs) and
-// one producer warp:
+// grid = (units, splits), one CTA per SM, 2 * np consumer warps (np pairs) and
+// one producer warp.  A unit is a KV head and up to 8 of its query heads (the
+// MMA's N): groups of more than 8 query heads per KV head run as several units
+// over the same cache (a second unit's reads of a tile mostly hit L2).
 //   setup    before the grid-dependency wait: the constant lookup tables (bulk
 //            copy; an L2 prefetch of the CTA's tiles there measured 8% slower
 //            over a 36-layer step).  After it: the head metadata, the key
 //            rotation blocks and the queries by bulk copy; q_rot = M_h q for
-//            the 8 query heads of the KV head, from each group's m x m block
+//            the unit's query heads, from each group's m x m block
 //            only, times log2(e) / (sqrt(d) sqrt(m_g)); its fp16 hi / lo MMA
 //            fragments.
 //   loop     the producer deals 7/8 of a head's tiles statically and the rest
@@ -91,7 +93,7 @@ struct DecodeArgs {
   const int32_t* block_table;  // [B][max_blocks] tile pages, or null: contiguous per head
   int64_t max_blocks;
   int q_fp32;
-  int hkv, gq;
+  int hkv, gq, nqs;  // KV heads per sequence, query heads per KV head, query slices
   int64_t T;
   int64_t n_tiles;    // capacity tiles per head (contiguous layout)
   int tile_bytes;
@@ -769,7 +771,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* stages = smem_raw + (stage_sa - raw_sa);
   const int area = (int)(kTabSharedAddr - stage_sa);  // bytes of the stage area
   float* pack = reinterpret_cast<float*>(stages + area - kPackArea);  // rotation pack at setup
-  const int head = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
+  // unit = (KV head, slice of at most kQSlice of its query heads); every unit
+  // streams its KV head's cache and keeps its own partials and tickets
+  const int unit = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
+  const int head = unit / a.nqs, qs = unit - head * a.nqs;
+  const int gq = min(kQSlice, a.gq - kQSlice * qs);  // query heads of this slice
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int np = a.np, ncw = 2 * np, S = a.ring;
   const bool producer = warp == ncw;
@@ -808,19 +814,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   pdl_wait();  // queries, metadata and the cache may come from the previous grid
   if (tid == 0) {
-    // the metadata, the first part of the rotation pack and the KV head's gq
+    // the metadata, the first part of the rotation pack and the unit's gq
     // queries (contiguous) land on one barrier; the queries go to qb as they are
-    const unsigned qbytes = (unsigned)(a.gq * kD * (a.q_fp32 ? 4 : 2));
+    const unsigned esz = a.q_fp32 ? 4u : 2u, qbytes = (unsigned)gq * kD * esz;
     mbar_expect_tx(&s.meta_bar, (unsigned)(sizeof(HeadMeta) + kPackPrefix) + qbytes);
     bulk_copy(&s.meta, a.meta + head, sizeof(HeadMeta), &s.meta_bar);
     bulk_copy(pack, a.rotpack + (size_t)head * kRotPackMaxWords, kPackPrefix, &s.meta_bar);
     bulk_copy(&s.qb[0][0],
-              reinterpret_cast<const uint8_t*>(a.q) + ((size_t)b * a.hkv + h) * qbytes, qbytes,
+              reinterpret_cast<const uint8_t*>(a.q) +
+                  (((size_t)b * a.hkv + h) * a.gq + (size_t)kQSlice * qs) * kD * esz,
+              qbytes,
               &s.meta_bar);
   }
   const int64_t T = a.seq_lens ? min((int64_t)a.seq_lens[b], a.T) : a.T;
   const int64_t tiles_T = (max(T, (int64_t)0) + kTile - 1) / kTile;
-  unsigned* head_tickets = a.tickets + (size_t)head * kTicketStride;
+  unsigned* head_tickets = a.tickets + (size_t)unit * kTicketStride;
   bool failed = false;
 
   // per-warp running state (consumers; set just before the tile loop)
@@ -991,13 +999,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < 8 * kD; i += nct) {
       const int p = i >> 3, hh = i & 7;
       float v = 0.f;
-      if (hh < a.gq && (p >> 1) < m.n_slots) {
+      if (hh < gq && (p >> 1) < m.n_slots) {
         const int d = (hh << 7) | (coord_dim[p] & (kD - 1));
         v = a.q_fp32 ? (&s.qb[0][0])[d] : __half2float(reinterpret_cast<const __half*>(&s.qb[0][0])[d]);
       }
       qT[p][hh] = v;
     }
-    if (split < n_w) window_fragments(s, a.q_fp32, a.gq, nct);  // before the rotation overwrites qb
+    if (split < n_w) window_fragments(s, a.q_fp32, gq, nct);  // before the rotation overwrites qb
     consumers_sync(nct);
     // q_rot[hh][pos] = sum_c R_g[r][c] qT[first + c][hh] * log2(e) / (sqrt(d) sqrt(m_g)),
     // into qb: a task is one position and four heads
@@ -1034,7 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (split < n_w) {
       const WindowArgs wa = {a.rk, a.rv, a.rs0, a.rs1, a.rs2};
       window_pass(wa, s, b, h, split, n_w, wl, ncw, reinterpret_cast<uint8_t*>(pack), smem_u32(pack),
-                  a.partials + ((size_t)head * a.slot_total + a.slot_window + split) * 8 * kPartialStride);
+                  a.partials + ((size_t)unit * a.slot_total + a.slot_window + split) * 8 * kPartialStride);
     }
     if (tid == 0) mbar_arrive(&s.done_bar);  // the pack's stages may be filled now
     // group descriptors: W | split << 4 | k16 tiles << 8 | half k-tile << 16
@@ -1312,7 +1320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
-  float* head_parts = a.partials + (size_t)head * a.slot_total * 8 * kPartialStride;
+  float* head_parts = a.partials + (size_t)unit * a.slot_total * 8 * kPartialStride;
   float* part = head_parts + (size_t)split * 8 * kPartialStride;
   // this CTA's (m, l, o_rot): the output itself with a single split, else its
   // partial in global memory; a task is 4 dims of one head
@@ -1407,10 +1415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     s.wl[0][tid] = cw;
   }
   __syncthreads();
-  float* out_head = a.out + ((size_t)b * a.hkv * a.gq + (size_t)h * a.gq) * kD;
+  float* out_head = a.out + (((size_t)b * a.hkv + h) * a.gq + (size_t)kQSlice * qs) * kD;
   auto window_o = [&](int hh, int dd) -> float { return n_w > 0 ? s.wl[0][hh] * s.qb[hh][dd] : 0.f; };
   if constexpr (VB == 0) {  // fp16 values: o_cache is already in the original basis
-    for (int idx = tid; idx < a.gq * kD; idx += blockDim.x) {
+    for (int idx = tid; idx < gq * kD; idx += blockDim.x) {
       const int hh = idx >> 7, dd = idx & (kD - 1);
       out_head[idx] = fmaf(s.wm[0][hh], s.qa[hh][dd], window_o(hh, dd));
     }
@@ -1447,7 +1455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int hh = 2 * t + (r & 1), d = dd + 8 * (r >> 1);
-      if (hh < a.gq) out_head[hh * kD + d] = fmaf(s.wm[0][hh], c[r], window_o(hh, d));
+      if (hh < gq) out_head[hh * kD + d] = fmaf(s.wm[0][hh], c[r], window_o(hh, d));
     }
   }
   }
@@ -1486,9 +1494,10 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   a.tickets = p->d_tickets;
   a.hkv = p->cfg.n_kv_heads;
   a.gq = p->g_q;
+  a.nqs = p->n_qs;
   a.dec_image = p->tab.dec_image;
   a.partials = p->d_partials;
-  const int split_cap = decode_split_cap(p->n_sms, p->n_heads);
+  const int split_cap = decode_split_cap(p->n_sms, p->n_units);
   const PartialSlots slots(split_cap);
   a.slot_groups = slots.groups;
   a.slot_window = slots.window;
@@ -1555,7 +1564,7 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   int splits = (int)std::min<int64_t>(split_cap, std::max<int64_t>(1, tiles_T));
   a.static_per = tiles_T * kStaticEighths / 8 / splits;
   cudaError_t e = cudaErrorInvalidValue;
-  const dim3 grid((unsigned)p->n_heads, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));
+  const dim3 grid((unsigned)p->n_units, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));
   switch (p->cfg.v_bits) {
 #define GTQ_LAUNCH_VB(VB)                                                                     \
   case VB:                                                                                   \

@@ -15,7 +15,8 @@ constexpr int kD = 128;                 // head_dim of quantize / decode
 constexpr int kBlocks = kD / 2;         // RoPE blocks per head
 constexpr int kMaxGroups = 8;           // one group per nonzero width 1..8
 constexpr int kMaxKt = 16;              // group-pure decode k-tiles: <= 8 + (groups - 1)
-constexpr int kMaxGq = 8;               // query heads per KV head handled by decode
+constexpr int kQSlice = 8;              // query heads one decode CTA serves (the MMA's N)
+constexpr int kMaxGq = 128;             // query heads per KV head (decode: slices of kQSlice)
 constexpr int kLutEntries = 510;        // sum over w = 1..8 of 2^w
 constexpr int kThrEntries = 502;        // sum over w = 1..8 of (2^w - 1)
 constexpr int kMaxSplits = 256;         // context splits per head in decode
@@ -210,6 +211,8 @@ struct gtq_plan {
   int n_heads;        // batch * n_kv_heads
   int n_blocks;       // head_dim / 2
   int g_q;            // n_q_heads / n_kv_heads
+  int n_qs;           // query slices per KV head: ceil(g_q / kQSlice)
+  int n_units;        // decode units: n_heads * n_qs (KV head, query slice) pairs
   int64_t n_tiles;    // tiles per head (capacity)
   size_t tile_bytes;
   size_t packed_bytes;
@@ -221,8 +224,8 @@ struct gtq_plan {
   float* d_mrow;      // [heads][128][128] key rotation rows in packed order (fp32)
   float* d_rotpack;   // [heads][kRotPackMaxWords] key rotation blocks for the decode kernel
   uint8_t* d_bimg;    // [heads] M_h as the quantizer's tensor-core B operand (64 KB each)
-  float* d_partials;  // [heads][PartialSlots(decode_split_cap).total][8][kPartialStride]
-  unsigned* d_tickets;  // [heads][kTicketStride] split-merge tickets and the tile counter
+  float* d_partials;  // [units][PartialSlots(decode_split_cap).total][8][kPartialStride]
+  unsigned* d_tickets;  // [units][kTicketStride] split-merge tickets and the tile counter
   int* d_status;      // device status word
 };
 

@@ -60,7 +60,7 @@ def _cfg(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(batch=0), gtq.GTQ_ERR_INVALID),
     (dict(n_q_heads=7), gtq.GTQ_ERR_INVALID),
-    (dict(n_q_heads=18), gtq.GTQ_ERR_UNSUPPORTED),      # GQA group of 9
+    (dict(n_q_heads=258), gtq.GTQ_ERR_UNSUPPORTED),     # GQA group of 129
     (dict(head_dim=130), gtq.GTQ_ERR_UNSUPPORTED),
     (dict(head_dim=12), gtq.GTQ_ERR_UNSUPPORTED),       # alloc from K needs a multiple of 8
     (dict(k_bits=0), gtq.GTQ_ERR_INVALID),

@@ -153,6 +153,7 @@ def check(case, check_codes=True):
     (1, 2, 7, 129, 4, 0),
     (1, 1, 1, 64, 3, 0),
     (1, 1, 8, 8192, 3, 0),     # several splits and both merge levels
+    (1, 2, 12, 900, 3, 0),     # a group of 12 query heads: units of 8 and 4
 ])
 def test_key_only_parity(B, hkv, gq, T, kb, pairing):
     check(Fp16Case(B, hkv, gq, T, kb, 0, pairing=pairing, seed=400 + T))
@@ -171,6 +172,13 @@ def test_window_parity(vb):
 @pytest.mark.parametrize("vb", [0, 2])
 def test_window_with_many_splits(vb):
     check(Fp16Case(1, 2, 8, 6000, 3, vb, W=300, seed=21 + vb))
+
+
+@pytest.mark.parametrize("vb", [0, 3])
+def test_window_with_large_query_groups(vb):
+    # 16 and 20 query heads per KV head with a window, ragged packed and window lengths
+    check(Fp16Case(2, 1, 16, 700, 3, vb, W=40, lens=[700, 130], wlens=[40, 9], seed=41 + vb))
+    check(Fp16Case(1, 2, 20, 2100, 2, vb, W=70, seed=43 + vb))
 
 
 def test_window_alone_is_plain_attention():

@@ -152,6 +152,13 @@ def check_case(case, check_decode=True, quantized=False):
     # wide tiles: fewer warp pairs per CTA, with enough tiles for two merge levels
     (1, 1, 8, 8192, 8, 8, 0, "fp16"),
     (2, 1, 4, 4000, 8, 6, 1, "fp16"),
+    # groups of more than 8 query heads: several units (8 query heads each) per KV
+    # head, the last one partial (9 = 8 + 1, 12 = 8 + 4), fp32 queries, and two
+    # merge levels per unit
+    (1, 1, 9, 333, 3, 2, 1, "fp16"),
+    (2, 2, 12, 1500, 3, 3, 0, "fp32"),
+    (1, 2, 16, 8192, 4, 4, 0, "fp16"),
+    (1, 1, 32, 4100, 2, 2, 0, "fp16"),
 ])
 def test_layer_parity(B, hkv, gq, T, kb, vb, pairing, dtype):
     check_case(Case(B, hkv, gq, T, kb, vb, pairing, dtype, seed=100 + T))
