@@ -459,7 +459,8 @@ def decode_variants(cfgd, w, dev, stream, hbm, steps, window=128, seed=7):
     captured in a CUDA graph and timed like the headline: a paged pool (pages
     in shuffled order, gtq_decode_attn_ex with a block table), K-only plans
     (keys coded, values read in fp16, gtq_decode_attn_full) and an fp16 window
-    of recent tokens beside the packed cache."""
+    of recent tokens beside the packed cache, and twice the query heads per KV
+    head."""
     import numpy as np
     import torch
 
@@ -555,6 +556,33 @@ def decode_variants(cfgd, w, dev, stream, hbm, steps, window=128, seed=7):
                          how="K%dV%d cache plus %d fp16 recent tokens per head in one softmax"
                              % (kb, vb, window))
     del g, rks, rvs, wkv
+    # ---- twice the query heads per KV head (two decode units of 8 per KV head)
+    plans2, q2, o2 = [], [], []
+    for layer, (k, _) in enumerate(w["kv"]):
+        cfg = gtq.make_config(B, 2 * hq, hkv, kb, vb, T)
+        with torch.cuda.stream(stream):
+            plans2.append(gtq.gtq_alloc_bits(cfg, k, T, stream=stream))
+        q2.append(w["qs"][layer].repeat(1, 2, 1))
+        o2.append(torch.empty((B, 2 * hq, 128), dtype=torch.float32, device=dev))
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    stream.synchronize()
+    # same keys, so the same allocation: the packed caches serve these plans too
+    same = all(np.array_equal(gtq.gtq_get_bits(p2), gtq.gtq_get_bits(p1))
+               for p1, p2 in zip(w["plans"], plans2))
+
+    def wide():
+        for layer in range(L):
+            gtq.gtq_decode_attn(plans2[layer], w["packed"][layer], T, q2[layer], o2[layer],
+                                stream=stream)
+
+    if same:
+        g = _graph_of(wide, stream)
+        ms = time_graph(g, steps, 3, stream)
+        out["q_group_x2"] = line(ms, w["step_bytes"], q_heads=2 * hq,
+                                 how="%d query heads per KV head (decode units of 8 query heads, "
+                                     "each streaming the KV head's cache)" % (2 * hq // hkv))
+        del g
+    del plans2, q2, o2
     torch.cuda.synchronize()
     return out
 
