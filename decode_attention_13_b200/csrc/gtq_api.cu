@@ -18,6 +18,8 @@ int check_config(const gtq_config* c, bool need_128) {
   if (!c) return GTQ_ERR_INVALID;
   if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1) return GTQ_ERR_INVALID;
   if (c->n_q_heads % c->n_kv_heads) return GTQ_ERR_INVALID;
+  // heads are the grid's y extent in the energy and quantize launches
+  if ((int64_t)c->batch * c->n_kv_heads > 65535) return GTQ_ERR_UNSUPPORTED;
   if (c->n_q_heads / c->n_kv_heads > kMaxGq) return GTQ_ERR_UNSUPPORTED;
   if (c->head_dim < 4 || c->head_dim > kD || (c->head_dim & 1)) return GTQ_ERR_UNSUPPORTED;
   if (need_128 && c->head_dim != kD) return GTQ_ERR_UNSUPPORTED;

@@ -88,7 +88,7 @@ typedef struct gtq_plan gtq_plan; /* opaque, library-owned */
 
 /* One layer's configuration.  Sizes in elements. */
 typedef struct gtq_config {
-  int32_t batch;        /* sequences B >= 1                                     */
+  int32_t batch;        /* sequences B >= 1; B * n_kv_heads <= 65535            */
   int32_t n_q_heads;    /* Hq, a multiple of n_kv_heads                         */
   int32_t n_kv_heads;   /* Hkv >= 1; Hq / Hkv (the GQA group) must be 1..128    */
   int32_t head_dim;     /* d: 128 for quantize/decode; any even 4..128 for alloc*/
@@ -116,7 +116,8 @@ typedef struct gtq_config {
  * Creates the plan, allocates its device memory (cudaMalloc; this call is not
  * capturable), and enqueues the energy, greedy and per-head metadata kernels.
  * Errors: INVALID (null, bad sizes/strides/alignment, bits out of range, Hq not
- * a multiple of Hkv), UNSUPPORTED (group > 128, head_dim not even 4..128), OOM, CUDA.
+ * a multiple of Hkv), UNSUPPORTED (group > 128, batch * Hkv > 65535, head_dim not
+ * even 4..128), OOM, CUDA.
  */
 GTQ_API int gtq_alloc_bits(const gtq_config* cfg, const void* k_dev, int64_t T,
                    const int64_t k_strides[4], void* stream, gtq_plan** out);

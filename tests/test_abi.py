@@ -61,6 +61,8 @@ def _cfg(**kw):
     (dict(batch=0), gtq.GTQ_ERR_INVALID),
     (dict(n_q_heads=7), gtq.GTQ_ERR_INVALID),
     (dict(n_q_heads=258), gtq.GTQ_ERR_UNSUPPORTED),     # GQA group of 129
+    (dict(batch=32768, n_q_heads=4), gtq.GTQ_ERR_UNSUPPORTED),  # 65536 KV heads
+    (dict(batch=1 << 30, n_q_heads=4), gtq.GTQ_ERR_UNSUPPORTED),  # int overflow of B * Hkv
     (dict(head_dim=130), gtq.GTQ_ERR_UNSUPPORTED),
     (dict(head_dim=12), gtq.GTQ_ERR_UNSUPPORTED),       # alloc from K needs a multiple of 8
     (dict(k_bits=0), gtq.GTQ_ERR_INVALID),
