@@ -31,14 +31,15 @@ inline int decode_split_cap(int n_sms, int n_heads) {
   const int s = n_heads >= 16 ? (n_sms + n_heads - 1) / n_heads : (n_sms / n_heads > 1 ? n_sms / n_heads : 1);
   return s < kMaxSplits ? s : kMaxSplits;
 }
-// Partial slots of one head: the splits, then the first-level group merges,
-// then the window partials.
+// Partial slots of one decode unit: the splits, then the first-level group
+// merges, then the window partials (one per split that attends window rows:
+// at most kWindowPartials and at most the splits).
 struct PartialSlots {
   int groups, window, total;
   explicit PartialSlots(int split_cap)
       : groups(split_cap),
         window(split_cap + (split_cap + kMergeGroup - 1) / kMergeGroup),
-        total(window + kWindowPartials) {}
+        total(window + (split_cap < kWindowPartials ? split_cap : kWindowPartials)) {}
 };
 constexpr int kMaxWindow = 1024;                // fp16 window rows per head (at most)
 constexpr int kStatusOverflow = 1;      // status word bits

@@ -181,6 +181,15 @@ def test_window_with_large_query_groups(vb):
     check(Fp16Case(1, 2, 20, 2100, 2, vb, W=70, seed=43 + vb))
 
 
+@pytest.mark.parametrize("vb", [0, 3])
+def test_window_on_every_split_of_many_units(vb):
+    # 16 decode units (4 x 4 KV heads; 2 x 4 KV heads x 2 query slices): 10
+    # splits each, and windows long enough (>= 10 blocks of 32 rows) that every
+    # split attends window rows, filling every window partial slot of a unit
+    check(Fp16Case(4, 4, 4, 1000, 3, vb, W=400, seed=51 + vb))
+    check(Fp16Case(2, 4, 12, 900, 2, vb, W=333, wlens=[333, 100], seed=53 + vb))
+
+
 def test_window_alone_is_plain_attention():
     # packed part empty in one sequence, window empty in another, both empty in a third
     check(Fp16Case(3, 1, 4, 200, 3, 3, W=50, lens=[0, 200, 0], wlens=[50, 0, 0], seed=31))
