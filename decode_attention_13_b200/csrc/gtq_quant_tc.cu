@@ -918,19 +918,37 @@ cudaError_t launch_quantize_tc(const gtq_plan* p, const void* k, const void* v, 
   // (a key tile costs about twice a value tile); every CTA keeps one head
   const int per_head = std::max(2, p->n_sms / std::max(1, p->n_heads));
   // The head's CTAs split between the roles (rounded share, at least one each),
-  // key and value CTAs together within the head's share of the SMs.  With only
-  // two per head (many heads) a head gets a third: two key CTAs and one value
-  // CTA, since a key tile costs about twice a value tile; the extra CTAs take
-  // the SMs that free up first (measured 10% faster than one of each).
-  const int share_k =
-      per_head == 2 ? 2 : std::min(per_head - 1, std::max(1, (per_head * kKeyShare + 50) / 100));
-  const int share_v = per_head == 2 ? 1 : per_head - share_k;
-  a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_k));
-  a.ctas_v = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_v));
-  if (p->cfg.v_bits == 0) {  // K-only: every CTA of the head codes keys
-    a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, per_head));
-    a.ctas_v = 0;
+  // key and value CTAs together within the head's share of the SMs.
+  const bool konly = p->cfg.v_bits == 0;
+  int share_k = std::min(per_head - 1, std::max(1, (per_head * kKeyShare + 50) / 100));
+  int share_v = per_head - share_k;
+  if (konly) {  // K-only: every CTA of the head codes keys
+    share_k = per_head;
+    share_v = 0;
   }
+  if (per_head == 2) {
+    // Many heads (fewer than three SMs each): each head takes 2u key CTAs and u
+    // value CTAs (u key CTAs alone for K-only plans), since a key tile costs
+    // about twice a value tile; the CTAs run in waves over the SMs.  u minimises
+    // the estimated finish: waves x (the busiest CTA's tiles in value-tile units
+    // + a set-up of about two value tiles).
+    int best_u = 1;
+    int64_t best = INT64_MAX;
+    for (int u = 1; u <= 8; ++u) {
+      const int ck = konly ? u : 2 * u, cv = konly ? 0 : u;
+      const int64_t waves = ((int64_t)p->n_heads * (ck + cv) + p->n_sms - 1) / p->n_sms;
+      const int64_t kt = (n_mt + ck - 1) / ck, vt = cv ? (n_mt + cv - 1) / cv : 0;
+      const int64_t est = waves * (std::max(2 * kt, vt) + 2);
+      if (est < best) {
+        best = est;
+        best_u = u;
+      }
+    }
+    share_k = konly ? best_u : 2 * best_u;
+    share_v = konly ? 0 : best_u;
+  }
+  a.ctas_k = (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_k));
+  a.ctas_v = konly ? 0 : (int)std::max<int64_t>(1, std::min<int64_t>(n_mt, share_v));
   cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
   if (e != cudaSuccess) return e;

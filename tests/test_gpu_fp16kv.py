@@ -159,6 +159,12 @@ def test_key_only_parity(B, hkv, gq, T, kb, pairing):
     check(Fp16Case(B, hkv, gq, T, kb, 0, pairing=pairing, seed=400 + T))
 
 
+def test_key_only_many_heads():
+    # 52 heads, fewer than three SMs each: K-only plans deal every head's key
+    # tiles to several CTAs that run in waves
+    check(Fp16Case(13, 4, 2, 1700, 3, 0, seed=63))
+
+
 def test_key_only_ragged_sequences():
     # rows past each length are NaN in the caller's value tensor; an empty sequence
     check(Fp16Case(3, 2, 4, 700, 3, 0, lens=[700, 65, 0], seed=7))

@@ -164,6 +164,12 @@ def test_layer_parity(B, hkv, gq, T, kb, vb, pairing, dtype):
     check_case(Case(B, hkv, gq, T, kb, vb, pairing, dtype, seed=100 + T))
 
 
+def test_many_heads_quantize_split():
+    # 64 heads, fewer than three SMs each: the quantizer deals every head's tiles
+    # to 2u key CTAs and u value CTAs (u = 2 here) that run in waves
+    check_case(Case(16, 4, 2, 2560, 3, 2, seed=61))
+
+
 @pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129])
 def test_ragged_lengths(T):
     check_case(Case(1, 2, 4, T, 3, 3, seed=T))
