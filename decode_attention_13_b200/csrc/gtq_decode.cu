@@ -1562,7 +1562,10 @@ cudaError_t launch_decode(const gtq_plan* p, const uint8_t* packed, int64_t T, c
   // one CTA per SM; with many heads, round up so that late CTAs join heads that
   // still have tiles left (the counter balances the work within a head)
   int splits = (int)std::min<int64_t>(split_cap, std::max<int64_t>(1, tiles_T));
-  a.static_per = tiles_T * kStaticEighths / 8 / splits;
+  // more CTAs than SMs: the last ones start a wave late, so every tile goes out
+  // by the counter (a static share of theirs would finish a wave late)
+  const bool waves = (int64_t)p->n_units * splits > p->n_sms;
+  a.static_per = waves ? 0 : tiles_T * kStaticEighths / 8 / splits;
   cudaError_t e = cudaErrorInvalidValue;
   const dim3 grid((unsigned)p->n_units, (unsigned)splits), block((unsigned)((2 * np + 1) * 32));
   switch (p->cfg.v_bits) {
