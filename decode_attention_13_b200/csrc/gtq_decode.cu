@@ -14,7 +14,8 @@
 //            only, times log2(e) / (sqrt(d) sqrt(m_g)); its fp16 hi / lo MMA
 //            fragments.
 //   loop     the producer deals 7/8 of a head's tiles statically and the rest
-//            from a per-head counter (two at a time, the next grab in flight),
+//            from a per-head counter (two at a time, the next grab in flight;
+//            every tile by the counter when the CTAs outnumber the SMs),
 //            and bulk-copies two adjacent 64-token tiles per stage into a ring;
 //            the pair that owns a tile splits it, 32 tokens per warp.  Scores:
 //            mma.m16n8k16 (m16n8k8 for a group's last half k-tile) with

@@ -8,8 +8,9 @@
 // one group of 128 and R_V.
 //
 // One launch; a CTA works on one head in one role, keys or values (about two
-// thirds of a head's CTAs take keys, whose tiles cost more), and walks the
-// 128-token tiles that lie inside the tokens being written.  Per tile:
+// thirds of a head's CTAs take keys, whose tiles cost more; with many heads,
+// 2u key and u value CTAs per head that run in waves), and walks the 128-token
+// tiles that lie inside the tokens being written.  Per tile:
 //   * code GEMM   D_c[coord][token] = R . X^T with R = M_h (keys) or R_V (values)
 //                 split into fp16 hi + lo parts (A operand, resident in shared
 //                 memory) and X the fp16 tile (B operand, TMA, 128B swizzle);
